@@ -1,0 +1,207 @@
+"""Causal softmax attention by its definition, in fp64 (oracle; test
+infrastructure only).
+
+Forward, for every global row i and query head h, kv head kh = floor(h*Hkv/Hq):
+    s_ij   = (q_i . k_j) * scale          for j <= i   (scale = 1/sqrt(d))
+    LSE_i  = ln sum_{j<=i} exp(s_ij)
+    O_i    = sum_{j<=i} exp(s_ij - LSE_i) v_j
+Scale and (B,S,H,D) layout: "LongVILA Guide" (aifetchly), section
+"Implementation", ``LongVILAMultiModalAttention.forward`` (scores divided by
+head_dim ** 0.5; q/k/v viewed as (b, s, n_heads, head_dim)). The ring method
+reaches exactly this result (up to rounding order), so the oracle does not
+simulate the ring for forward parity; ``merge.ring_attention`` does, to pin
+the merge.
+
+Backward (the pages give none; a reading: the gradient of the definition
+above), with P_ij = exp(s_ij - LSE_i) and D_i = sum_d dO_i * O_i:
+    dV_j = sum_i P_ij dO_i            (summed over the q heads of kv head kh)
+    dP_ij = dO_i . v_j
+    dS_ij = P_ij (dP_ij - D_i)
+    dQ_i = scale sum_j dS_ij k_j
+    dK_j = scale sum_i dS_ij q_i      (summed over the q heads of kv head kh)
+
+Inputs are numpy arrays (any float dtype; converted to fp64) of shape
+[N, H, d]. Rows are processed in blocks only to bound memory; every block is
+the plain formula.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+NEG_INF = -np.inf
+
+
+def kv_head(h: int, hq: int, hkv: int) -> int:
+    """GQA mapping (reading): contiguous groups of Hq/Hkv query heads."""
+    return (h * hkv) // hq
+
+
+def _f64(x):
+    if hasattr(x, "detach"):
+        x = x.detach().float().cpu().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def _rows_forward(qr, rows, K, V, scale):
+    """O and LSE for query vectors qr [R,d] at global positions rows [R]
+    against keys K[:i+1], V[:i+1] (one head)."""
+    R = len(rows)
+    d = V.shape[1]
+    O = np.zeros((R, d))
+    L = np.full(R, NEG_INF)
+    if R == 0:
+        return O, L
+    jmax = int(rows.max()) + 1
+    s = (qr @ K[:jmax].T) * scale                      # [R, jmax]
+    visible = np.arange(jmax)[None, :] <= rows[:, None]
+    s = np.where(visible, s, NEG_INF)
+    m = s.max(axis=1)
+    lse = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+    p = np.exp(s - lse[:, None])                        # 0 where masked
+    O = p @ V[:jmax]
+    return O, lse
+
+
+def causal_attention(q, k, v, scale=None, block: int = 512):
+    """Whole-sequence forward. Returns (O [N,Hq,d], LSE [N,Hq]) in fp64."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    N, hq, d = q.shape
+    hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    O = np.zeros((N, hq, d))
+    LSE = np.zeros((N, hq))
+    for h in range(hq):
+        kh = kv_head(h, hq, hkv)
+        for i0 in range(0, N, block):
+            rows = np.arange(i0, min(N, i0 + block))
+            o, l = _rows_forward(q[rows, h], rows, k[:, kh], v[:, kh], scale)
+            O[rows, h] = o
+            LSE[rows, h] = l
+    return O, LSE
+
+
+def attention_rows(q, k, v, rows, scale=None, block: int = 64):
+    """Forward for selected global rows only. Returns (O [R,Hq,d], LSE [R,Hq])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    rows = np.asarray(rows, np.int64)
+    N, hq, d = q.shape
+    hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    O = np.zeros((len(rows), hq, d))
+    LSE = np.zeros((len(rows), hq))
+    for h in range(hq):
+        kh = kv_head(h, hq, hkv)
+        for b0 in range(0, len(rows), block):
+            sel = np.arange(b0, min(len(rows), b0 + block))
+            o, l = _rows_forward(q[rows[sel], h], rows[sel], k[:, kh], v[:, kh], scale)
+            O[sel, h] = o
+            LSE[sel, h] = l
+    return O, LSE
+
+
+def _rows_backward(qr, dor, rows, K, V, scale):
+    """For one head and query rows: (O, LSE, D, dQ rows, P, dS) restricted to
+    keys [0, max(rows)]; P and dS are [R, jmax]."""
+    jmax = int(rows.max()) + 1
+    s = (qr @ K[:jmax].T) * scale
+    visible = np.arange(jmax)[None, :] <= rows[:, None]
+    s = np.where(visible, s, NEG_INF)
+    m = s.max(axis=1)
+    lse = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+    p = np.exp(s - lse[:, None])
+    o = p @ V[:jmax]
+    D = (dor * o).sum(axis=1)
+    dp = dor @ V[:jmax].T
+    ds = p * (dp - D[:, None])
+    dq = scale * (ds @ K[:jmax])
+    return o, lse, D, dq, p, ds
+
+
+def causal_attention_bwd(q, k, v, do, scale=None, block: int = 512):
+    """Whole-sequence backward of the definition.
+
+    Returns dict with O, LSE, D [N,Hq], dQ [N,Hq,d], dK, dV [N,Hkv,d] (fp64).
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    N, hq, d = q.shape
+    hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    O = np.zeros((N, hq, d))
+    LSE = np.zeros((N, hq))
+    Dm = np.zeros((N, hq))
+    dQ = np.zeros((N, hq, d))
+    dK = np.zeros((N, hkv, d))
+    dV = np.zeros((N, hkv, d))
+    for h in range(hq):
+        kh = kv_head(h, hq, hkv)
+        for i0 in range(0, N, block):
+            rows = np.arange(i0, min(N, i0 + block))
+            o, lse, D, dq, p, ds = _rows_backward(q[rows, h], do[rows, h], rows,
+                                                  k[:, kh], v[:, kh], scale)
+            jmax = p.shape[1]
+            O[rows, h] = o
+            LSE[rows, h] = lse
+            Dm[rows, h] = D
+            dQ[rows, h] = dq
+            dV[:jmax, kh] += p.T @ do[rows, h]
+            dK[:jmax, kh] += scale * (ds.T @ q[rows, h])
+    return {"O": O, "LSE": LSE, "D": Dm, "dQ": dQ, "dK": dK, "dV": dV}
+
+
+def attention_bwd_rows(q, k, v, do, rows, scale=None, block: int = 64):
+    """dQ (and O, LSE) for selected global rows: row i needs only keys <= i."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    rows = np.asarray(rows, np.int64)
+    N, hq, d = q.shape
+    hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    R = len(rows)
+    dQ = np.zeros((R, hq, d))
+    O = np.zeros((R, hq, d))
+    LSE = np.zeros((R, hq))
+    for h in range(hq):
+        kh = kv_head(h, hq, hkv)
+        for b0 in range(0, R, block):
+            sel = np.arange(b0, min(R, b0 + block))
+            o, lse, _, dq, _, _ = _rows_backward(q[rows[sel], h], do[rows[sel], h], rows[sel],
+                                                 k[:, kh], v[:, kh], scale)
+            dQ[sel, h] = dq
+            O[sel, h] = o
+            LSE[sel, h] = lse
+    return {"O": O, "LSE": LSE, "dQ": dQ}
+
+
+def attention_bwd_keys(q, k, v, do, keys, scale=None, block: int = 64):
+    """dK and dV for selected global key positions.
+
+    Key j receives contributions from rows i >= j only, so this computes the
+    rows [min(keys), N) in full (their LSE and D) and sums their terms into
+    the requested keys. Cheap only when the keys lie near the end.
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    keys = np.asarray(keys, np.int64)
+    N, hq, d = q.shape
+    hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    j0 = int(keys.min())
+    dK = np.zeros((len(keys), hkv, d))
+    dV = np.zeros((len(keys), hkv, d))
+    for h in range(hq):
+        kh = kv_head(h, hq, hkv)
+        for i0 in range(j0, N, block):
+            rows = np.arange(i0, min(N, i0 + block))
+            _, _, _, _, p, ds = _rows_backward(q[rows, h], do[rows, h], rows,
+                                               k[:, kh], v[:, kh], scale)
+            pk = p[:, keys[keys <= rows.max()]]
+            dsk = ds[:, keys[keys <= rows.max()]]
+            sel = np.nonzero(keys <= rows.max())[0]
+            dV[sel, kh] += pk.T @ do[rows, h]
+            dK[sel, kh] += scale * (dsk.T @ q[rows, h])
+    return {"dK": dK, "dV": dV}

@@ -1,0 +1,33 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that the pins
+catch them: a pin that cannot fail pins nothing."""
+import numpy as np
+import pytest
+
+from conftest import load_golden
+from oracle import attention as A
+from oracle import merge as M
+import test_oracle_attention as TA
+
+
+def test_interleaved_gqa_mapping_is_caught(monkeypatch):
+    monkeypatch.setattr(A, "kv_head", lambda h, hq, hkv: h % hkv)
+    with pytest.raises(AssertionError):
+        TA.test_hand_worked_example()
+
+
+def test_wrong_scale_is_caught(monkeypatch):
+    real = A._rows_forward
+    monkeypatch.setattr(A, "_rows_forward",
+                        lambda qr, rows, K, V, scale: real(qr, rows, K, V, scale * 2.0))
+    with pytest.raises(AssertionError):
+        TA.test_matches_torch_sdpa_fp64(37, 4, 4, 16)
+
+
+def test_dropped_merge_weight_is_caught():
+    g = load_golden("merge_hand.txt")
+    oa, ob = np.array(g["o_a"]), np.array(g["o_b"])
+    # the page's sketch: plain sum of the normalised blocks
+    wrong = oa + ob
+    assert not np.allclose(wrong, g["o_out"])
+    o, _ = M.lse_merge(oa, g["lse_a"][0], ob, g["lse_b"][0])
+    assert np.allclose(o, g["o_out"])
