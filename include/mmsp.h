@@ -1,0 +1,204 @@
+/*
+ * mmsp.h -- C ABI of libmmsp.so: ring-blockwise causal attention over a
+ * zigzag-sharded sequence of interleaved video and text tokens, with all P
+ * virtual ranks of the ring computed on one B200 (sm_100a).
+ *
+ * Method source: "LongVILA Guide: 2M Context Multi-Modal AI Model"
+ * (aifetchly blog), sections "Problem" (576 visual tokens per frame,
+ * interleaved text), "Multi-Modal Sequence Parallelism (MM-SP) Mechanics"
+ * (Ring-SP: each rank holds N/P tokens, K/V blocks travel around the ring in
+ * P-1 shifts) and "Implementation" (LongVILAParallelContext ring neighbours;
+ * LongVILAMultiModalAttention.forward: (B,S,H,D) layout, scores scaled by
+ * 1/sqrt(head_dim), per-step block attention). The log-sum-exp combine, the
+ * causal mask, zigzag sharding and GQA head grouping are readings of those
+ * passages (the page's sketch sums separately normalised blocks).
+ *
+ * Conventions for every entry point
+ *   - Returns an mmsp_status; MMSP_OK on success. On failure the message of
+ *     the calling thread's last error is available from mmsp_last_error().
+ *   - All arguments are validated on the host before anything is launched;
+ *     a rejected call launches nothing and touches no buffer.
+ *   - Device pointers are caller-owned (the library allocates no device
+ *     memory); host pointers are read during the call only.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t passed as
+ *     void*; NULL means the legacy default stream). Nothing synchronises.
+ *   - bf16 tensors are raw 16-bit bfloat16 words (const void*).
+ *   - Token-major layouts: a tensor "[T][H][d]" is row-major with d
+ *     contiguous; rank-local tensors are "[P][2C][H][d]" where C = N/(2P)
+ *     and rank r's local slot t holds global token
+ *         (t < C ? r*C + t : (2P-1-r)*C + (t-C))      (zigzag).
+ *   - LSE values are natural logarithms; a row with no visible key has
+ *     LSE = -inf and O = 0.
+ *   - Device-side waits are bounded; a wait that gives up records a timeout
+ *     that mmsp_device_status() reports as MMSP_ETIMEOUT. No kernel traps.
+ */
+#ifndef MMSP_H
+#define MMSP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MMSP_OK = 0,
+  MMSP_EINVAL = 1,       /* bad argument (size, alignment, NULL, layout) */
+  MMSP_EUNSUPPORTED = 2, /* valid request this build does not implement   */
+  MMSP_ECUDA = 3,        /* a CUDA runtime/driver call failed             */
+  MMSP_ETIMEOUT = 4      /* a bounded device-side wait gave up            */
+} mmsp_status;
+
+/* flags for mmsp_attn_fwd */
+#define MMSP_ACCUMULATE 1u /* merge into the running (o_acc, lse) state   */
+#define MMSP_FINALIZE 2u   /* also write o_out = bf16(o_acc) (RNE)         */
+
+#define MMSP_MAX_SEGMENTS 4096 /* capacity of the segment table per call */
+
+/*
+ * mmsp_shard -- the zigzag shard step: index maps and an optional row permute.
+ *
+ * Source: "LongVILA Guide", section "MM-SP Mechanics", Ring-SP paragraph
+ * (each rank holds N/P tokens), and LongVILAMultiModalAttention.forward's
+ * docstring (local length = total / number of ranks). Zigzag (rank r owns
+ * chunks r and 2P-1-r of 2P equal chunks) is a reading that balances causal
+ * work across ranks.
+ *
+ *   seg_len, seg_kind  HOST arrays of n_seg entries: the packed sequence as
+ *                      segments in order (kind 0 = text, 1 = visual; frames
+ *                      are 576-token visual segments). Must sum to N.
+ *                      May be NULL (with n_seg = 0) when none of
+ *                      modality_local / segid_local / rank_counts is wanted.
+ *   N, P               tokens and virtual ranks; N % (2P) == 0, N < 2^31.
+ *   local2global       DEVICE int32[N] or NULL: global position of local slot.
+ *   global2local       DEVICE int32[N] or NULL: inverse permutation.
+ *   modality_local     DEVICE uint8[N] or NULL: kind of each local slot.
+ *   segid_local        DEVICE int32[N] or NULL: segment index of each slot.
+ *   rank_counts        DEVICE int32[P][2] or NULL: text, visual counts per rank.
+ *   src, dst           DEVICE row buffers or both NULL. With inverse == 0:
+ *                      dst[l] = src[local2global(l)] (global -> rank-local);
+ *                      with inverse != 0: dst[local2global(l)] = src[l].
+ *                      Rows are row_bytes long; src, dst and row_bytes must be
+ *                      multiples of 16 bytes; src and dst must not overlap.
+ * Bit-exact: pure integer / byte work.
+ */
+int mmsp_shard(const int32_t* seg_len, const uint8_t* seg_kind, int32_t n_seg,
+               int64_t N, int32_t P,
+               int32_t* local2global, int32_t* global2local,
+               uint8_t* modality_local, int32_t* segid_local, int32_t* rank_counts,
+               const void* src, void* dst, int64_t row_bytes, int32_t inverse,
+               void* stream);
+
+/*
+ * mmsp_attn_fwd -- blockwise causal attention of every virtual rank's queries
+ * over the K/V blocks it holds at ring steps [step_begin, step_end), merged
+ * across steps with the online-softmax (log-sum-exp) combine.
+ *
+ * Source: "LongVILA Guide", section "Implementation",
+ * LongVILAMultiModalAttention.forward (ring loop over ring_size steps; block
+ * attention on the current K/V; scores * 1/sqrt(head_dim)) and
+ * LongVILAParallelContext (receive from the previous ring rank): at step s,
+ * rank r holds the K/V of rank (r - s) mod P.
+ *
+ *   q                  DEVICE bf16 [P][2C][Hq][d]  rank-local queries
+ *   k, v               DEVICE bf16 [P][2C][Hkv][d] rank-local keys/values
+ *   N, P, Hq, Hkv, d   N % (2P) == 0; Hq % Hkv == 0; d in {64, 128}.
+ *                      Query head h reads kv head floor(h*Hkv/Hq).
+ *   scale              softmax scale (1/sqrt(d) for the pages' layer).
+ *   causal             1: key j visible to query i iff global j <= global i;
+ *                      0: every key visible.
+ *   step_begin/end     0 <= begin <= end <= P; (0, P) is the whole ring.
+ *   o_acc              DEVICE fp32 [P][2C][Hq][d]: normalised output over the
+ *                      keys seen so far. Read when flags has MMSP_ACCUMULATE,
+ *                      written when non-NULL. Required with MMSP_ACCUMULATE.
+ *   lse                DEVICE fp32 [P][2C][Hq]: running LSE (natural log).
+ *                      Read with MMSP_ACCUMULATE; always written.
+ *   o_out              DEVICE bf16 [P][2C][Hq][d]: written (round to nearest
+ *                      even) when flags has MMSP_FINALIZE; else may be NULL.
+ *   flags              MMSP_ACCUMULATE | MMSP_FINALIZE.
+ * Without MMSP_ACCUMULATE the state starts empty (LSE -inf, O 0).
+ * All pointers 16-byte aligned. fp32 accumulation; tcgen05 tensor cores.
+ */
+int mmsp_attn_fwd(const void* q, const void* k, const void* v,
+                  int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d,
+                  float scale, int32_t causal,
+                  int32_t step_begin, int32_t step_end,
+                  float* o_acc, float* lse, void* o_out,
+                  uint32_t flags, void* stream);
+
+/*
+ * mmsp_lse_merge -- combine two partial attention results over disjoint key
+ * sets (the per-step combine of the ring; replaces the page's plain sum of
+ * normalised blocks in the ring loop of LongVILAMultiModalAttention.forward):
+ *   m = max(la, lb); L = m + ln(e^(la-m) + e^(lb-m));
+ *   O = e^(la-L) Oa + e^(lb-L) Ob;   both -inf -> (O, L) = (0, -inf).
+ *
+ *   o_a, o_b, o_out    DEVICE fp32 [rows][H][d]; o_out may equal o_a or o_b.
+ *   lse_a, lse_b, lse_out DEVICE fp32 [rows][H]; lse_out may equal an input.
+ *   rows, H, d         d in {4, 8, 16, 32, 64, 128}. o pointers 16-byte
+ *                      aligned, lse pointers 4-byte aligned.
+ */
+int mmsp_lse_merge(const float* o_a, const float* lse_a,
+                   const float* o_b, const float* lse_b,
+                   float* o_out, float* lse_out,
+                   int64_t rows, int32_t H, int32_t d, void* stream);
+
+/*
+ * mmsp_attn_bwd -- gradients of the ring attention (whole ring, all P ranks).
+ *
+ * The pages give only the backward of the all-to-all transpose; this is a
+ * reading: the gradient of causal softmax attention, with P_ij = exp(s_ij -
+ * LSE_i) recomputed from the saved fp32 LSE and D_i = sum_d dO_i * O_i:
+ *   dV_j = sum_i P_ij dO_i;  dS_ij = P_ij (dO_i . v_j - D_i);
+ *   dQ_i = scale sum_j dS_ij k_j;  dK_j = scale sum_i dS_ij q_i;
+ * dK and dV sum over the Hq/Hkv query heads of each kv head.
+ *
+ *   q, k, v, o, dout   DEVICE bf16, rank-local, shapes as in mmsp_attn_fwd.
+ *   lse                DEVICE fp32 [P][2C][Hq] from mmsp_attn_fwd (whole ring).
+ *   dq                 DEVICE bf16 [P][2C][Hq][d]  (output)
+ *   dk, dv             DEVICE bf16 [P][2C][Hkv][d] (output)
+ *   dq_acc_opt         DEVICE fp32 [P][2C][Hq][d] or NULL: fp32 dQ output.
+ *   workspace          DEVICE scratch of at least mmsp_bwd_workspace_bytes()
+ *                      bytes, 256-byte aligned; contents need not be zeroed.
+ *   d == 128 or 64; other constraints as mmsp_attn_fwd.
+ */
+int mmsp_attn_bwd(const void* q, const void* k, const void* v,
+                  const void* o, const void* dout, const float* lse,
+                  int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d,
+                  float scale, int32_t causal,
+                  void* dq, void* dk, void* dv, float* dq_acc_opt,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Scratch bytes mmsp_attn_bwd needs for these sizes (0 on invalid sizes). */
+size_t mmsp_bwd_workspace_bytes(int64_t N, int32_t P, int32_t Hq, int32_t d);
+
+/* Message of the calling thread's last failed call ("" if none). */
+const char* mmsp_last_error(void);
+
+/*
+ * mmsp_device_status -- synchronise `stream`, then report (and clear) a
+ * bounded-wait timeout recorded by any kernel of this library on the current
+ * device since the previous call: MMSP_ETIMEOUT if one was recorded,
+ * MMSP_ECUDA on a CUDA error, else MMSP_OK.
+ */
+int mmsp_device_status(void* stream);
+
+/*
+ * mmsp_selftest_bounded_wait -- launch one CTA that waits on an mbarrier no
+ * one arrives on, using the same bounded wait as the attention kernels, with
+ * a cap of max_cycles SM clock cycles; the kernel records a timeout and
+ * returns. Used by the tests to show that a wait that cannot finish ends with
+ * MMSP_ETIMEOUT from mmsp_device_status() instead of hanging.
+ * max_cycles in [1, 2^31].
+ */
+int mmsp_selftest_bounded_wait(int64_t max_cycles, void* stream);
+
+/* Library version string. */
+const char* mmsp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MMSP_H */

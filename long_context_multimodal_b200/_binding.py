@@ -1,0 +1,154 @@
+"""ctypes marshalling for libmmsp.so. Same names and argument order as the C
+ABI in include/mmsp.h; tensors are passed by device pointer."""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import c_float, c_int32, c_int64, c_size_t, c_uint32, c_void_p
+
+import numpy as np
+
+MMSP_ACCUMULATE = 1
+MMSP_FINALIZE = 2
+MMSP_MAX_SEGMENTS = 4096
+STATUS = {0: "MMSP_OK", 1: "MMSP_EINVAL", 2: "MMSP_EUNSUPPORTED", 3: "MMSP_ECUDA", 4: "MMSP_ETIMEOUT"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def lib_path() -> str:
+    return os.path.join(_HERE, "libmmsp.so")
+
+
+class MmspError(RuntimeError):
+    def __init__(self, func: str, status: int, message: str):
+        self.status = status
+        super().__init__(f"{func} -> {STATUS.get(status, status)}: {message}")
+
+
+def _load():
+    path = lib_path()
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing: build the CUDA library first "
+            "(python -m long_context_multimodal_b200.build). There is no CPU fallback.")
+    return ctypes.CDLL(path)
+
+
+_lib = _load()
+
+_SIGS = {
+    "mmsp_shard": ([c_void_p, c_void_p, c_int32, c_int64, c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
+                    c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_void_p], c_int32),
+    "mmsp_attn_fwd": ([c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32, c_int32, c_int32, c_float,
+                       c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_uint32, c_void_p], c_int32),
+    "mmsp_lse_merge": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32,
+                        c_void_p], c_int32),
+    "mmsp_attn_bwd": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32,
+                       c_int32, c_int32, c_float, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                       c_size_t, c_void_p], c_int32),
+    "mmsp_bwd_workspace_bytes": ([c_int64, c_int32, c_int32, c_int32], c_size_t),
+    "mmsp_last_error": ([], ctypes.c_char_p),
+    "mmsp_device_status": ([c_void_p], c_int32),
+    "mmsp_selftest_bounded_wait": ([c_int64, c_void_p], c_int32),
+    "mmsp_version": ([], ctypes.c_char_p),
+}
+for _name, (_args, _ret) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = _ret
+
+
+def exported_symbols():
+    """Names of the C ABI this binding declares (all must resolve in the .so)."""
+    return list(_SIGS)
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        if not x.is_contiguous():
+            raise ValueError("tensor arguments must be contiguous")
+        return x.data_ptr()
+    raise TypeError(f"expected a tensor, an int pointer or None, got {type(x)}")
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+
+        if torch.cuda.is_available():
+            return torch.cuda.current_stream().cuda_stream
+        return None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(name, rc):
+    if rc != 0:
+        raise MmspError(name, rc, _lib.mmsp_last_error().decode())
+    return rc
+
+
+def mmsp_last_error() -> str:
+    return _lib.mmsp_last_error().decode()
+
+
+def mmsp_version() -> str:
+    return _lib.mmsp_version().decode()
+
+
+def mmsp_shard(seg_len, seg_kind, N, P, local2global=None, global2local=None, modality_local=None,
+               segid_local=None, rank_counts=None, src=None, dst=None, row_bytes=0, inverse=False, stream=None):
+    """Index maps and/or row permute of the zigzag shard step (see mmsp.h)."""
+    n_seg = 0
+    sl = sk = None
+    if seg_len is not None:
+        sl_arr = np.ascontiguousarray(np.asarray(seg_len, dtype=np.int32))
+        sk_arr = np.ascontiguousarray(np.asarray(seg_kind, dtype=np.uint8))
+        n_seg = int(sl_arr.size)
+        sl = sl_arr.ctypes.data_as(c_void_p)
+        sk = sk_arr.ctypes.data_as(c_void_p)
+    rc = _lib.mmsp_shard(sl, sk, n_seg, int(N), int(P), _ptr(local2global), _ptr(global2local),
+                         _ptr(modality_local), _ptr(segid_local), _ptr(rank_counts), _ptr(src), _ptr(dst),
+                         int(row_bytes), int(bool(inverse)), _stream(stream))
+    return _check("mmsp_shard", rc)
+
+
+def mmsp_attn_fwd(q, k, v, N, P, Hq, Hkv, d, scale, causal, step_begin, step_end, o_acc, lse, o_out,
+                  flags, stream=None):
+    rc = _lib.mmsp_attn_fwd(_ptr(q), _ptr(k), _ptr(v), int(N), int(P), int(Hq), int(Hkv), int(d), float(scale),
+                            int(causal), int(step_begin), int(step_end), _ptr(o_acc), _ptr(lse), _ptr(o_out),
+                            int(flags), _stream(stream))
+    return _check("mmsp_attn_fwd", rc)
+
+
+def mmsp_lse_merge(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, H, d, stream=None):
+    rc = _lib.mmsp_lse_merge(_ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(o_out), _ptr(lse_out),
+                             int(rows), int(H), int(d), _stream(stream))
+    return _check("mmsp_lse_merge", rc)
+
+
+def mmsp_attn_bwd(q, k, v, o, dout, lse, N, P, Hq, Hkv, d, scale, causal, dq, dk, dv, dq_acc_opt,
+                  workspace, workspace_bytes, stream=None):
+    rc = _lib.mmsp_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), int(N), int(P), int(Hq),
+                            int(Hkv), int(d), float(scale), int(causal), _ptr(dq), _ptr(dk), _ptr(dv),
+                            _ptr(dq_acc_opt), _ptr(workspace), int(workspace_bytes), _stream(stream))
+    return _check("mmsp_attn_bwd", rc)
+
+
+def mmsp_bwd_workspace_bytes(N, P, Hq, d) -> int:
+    return int(_lib.mmsp_bwd_workspace_bytes(int(N), int(P), int(Hq), int(d)))
+
+
+def mmsp_device_status(stream=None) -> int:
+    """Synchronise the stream; raises MmspError on a recorded timeout."""
+    return _check("mmsp_device_status", _lib.mmsp_device_status(_stream(stream)))
+
+
+def mmsp_selftest_bounded_wait(max_cycles, stream=None):
+    return _check("mmsp_selftest_bounded_wait", _lib.mmsp_selftest_bounded_wait(int(max_cycles), _stream(stream)))

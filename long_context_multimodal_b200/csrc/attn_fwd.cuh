@@ -1,0 +1,569 @@
+// attn_fwd.cuh -- ring-blockwise causal attention forward on tcgen05 tensor
+// cores, all P virtual ranks of the ring in one persistent launch.
+//
+// Method: "LongVILA Guide" (aifetchly), section "Implementation",
+// LongVILAMultiModalAttention.forward: for ring_size steps each rank runs
+// block attention of its queries against the K/V block it currently holds
+// (scores scaled by 1/sqrt(head_dim)), then receives the next block from the
+// previous ring rank (LongVILAParallelContext, "Identify Ring Neighbors").
+// So rank r holds the K/V of rank (r - s) mod P at step s. The per-step
+// results are merged with the online-softmax (log-sum-exp) combine -- a
+// reading; the page's sketch sums normalised blocks -- which, carried in
+// registers/TMEM across the steps, is the fused form of mmsp_lse_merge.
+//
+// Work unit ("item"): one head h and 256 consecutive query rows (two 128-row
+// tiles A and B) of one zigzag chunk of one virtual rank. Items are ordered
+// by decreasing causal work (q chunk 2P-1 first), then kv head, row block,
+// query head, so CTAs running together stream the same K/V tiles through L2.
+// The CTA visits the item's K/V tiles of 128 keys in ring order and skips
+// (chunk, tile) pairs the causal mask empties.
+//
+// Warp roles (320 threads, one CTA per SM):
+//   warp 0      TMA producer: Q tiles A/B once per item, then K_j, V_j into
+//               a 3-stage ring of 128 x d bf16 tiles (128-byte swizzle).
+//   warp 1      MMA issuer (one thread): S_X = Q_X K_j^T into TMEM, and
+//               O_X += P_X V_j with P_X from shared memory; ping-pong order
+//               PV_A(j), S_A(j+1), PV_B(j), S_B(j+1) so the tensor core works
+//               on one tile while the softmax warps work on the other.
+//   warps 2-5   softmax for tile A, warps 6-9 for tile B: one thread per row
+//               (TMEM lane), fp32 online softmax in base 2, P written to
+//               shared memory as bf16, lazy O rescale (only when the running
+//               max grows by more than 2^8), epilogue O / l and LSE.
+// TMEM: S_A [0,128) S_B [128,256) O_A [256,256+d) O_B [256+d,256+2d).
+#pragma once
+
+#include <cuda.h>
+#include <math_constants.h>
+
+#include <type_traits>
+
+#include "ptx.cuh"
+
+namespace mmsp {
+namespace fwd {
+
+constexpr int BM = 128;      // query rows per tile
+constexpr int BN = 128;      // keys per tile
+constexpr int NSTAGE = 3;    // K/V ring stages
+constexpr int kThreads = 320;
+constexpr int HALF = 128 * 128;  // bytes of one 128-row x 64-column bf16 half tile
+
+struct Params {
+  int32_t P, Hq, Hkv, G;
+  int64_t C;        // zigzag chunk length N / (2P)
+  int32_t nblk;     // 256-row blocks per chunk
+  int32_t causal, step_begin, step_end;
+  int32_t accumulate, finalize;
+  int64_t n_items;
+  float scale_log2;  // softmax scale * log2(e)
+  float* o_acc;
+  float* lse;
+  __nv_bfloat16* o_out;
+  long long wait_cap;
+};
+
+struct Item {
+  int r, c, blk, h, kvh;
+  int64_t rowA0;       // first row of tile A within its chunk
+  bool validA, validB;
+};
+
+__device__ __forceinline__ Item decode_item(const Params& p, int64_t idx) {
+  const int64_t per_group = (int64_t)p.nblk * p.Hq;
+  const int g = (int)(idx / per_group);
+  const int64_t w = idx - (int64_t)g * per_group;
+  Item it;
+  // group g works on global query chunk 2P-1-g: chunk 1 of rank g for g < P,
+  // chunk 0 of rank 2P-1-g otherwise.
+  if (g < p.P) {
+    it.r = g;
+    it.c = 1;
+  } else {
+    it.r = 2 * p.P - 1 - g;
+    it.c = 0;
+  }
+  const int hg = (int)(w % p.G);
+  const int64_t w2 = w / p.G;
+  it.blk = (int)(w2 % p.nblk);
+  it.kvh = (int)(w2 / p.nblk);
+  it.h = it.kvh * p.G + hg;
+  it.rowA0 = (int64_t)it.blk * 256;
+  it.validA = it.rowA0 < p.C;
+  it.validB = it.rowA0 + 128 < p.C;
+  return it;
+}
+
+// Enumerates the K/V tiles an item visits, in ring order.
+struct TileIter {
+  int r, P, gq, causal, s, se, ck, t, tmax, ntiles;
+  int64_t C, rowA0, base_row;
+  bool validA, validB, in_chunk, diag;
+  // current tile
+  int64_t kv_row;
+  int key0;
+  bool actA, actB, maskA, maskB;
+
+  __device__ __forceinline__ TileIter(const Params& p, const Item& it) {
+    r = it.r;
+    P = p.P;
+    gq = it.c ? 2 * p.P - 1 - it.r : it.r;
+    causal = p.causal;
+    s = p.step_begin;
+    se = p.step_end;
+    ck = 0;
+    t = 0;
+    tmax = -1;
+    C = p.C;
+    ntiles = (int)((p.C + BN - 1) / BN);
+    rowA0 = it.rowA0;
+    validA = it.validA;
+    validB = it.validB;
+    in_chunk = false;
+    diag = false;
+  }
+
+  __device__ __forceinline__ bool next() {
+    while (true) {
+      if (!in_chunk) {
+        if (s >= se) return false;
+        int k = (r - s) % P;
+        if (k < 0) k += P;
+        const int gk = ck ? 2 * P - 1 - k : k;
+        const bool skip = causal && gk > gq;
+        diag = causal && gk == gq;
+        base_row = (int64_t)k * 2 * C + (int64_t)ck * C;
+        if (++ck == 2) {
+          ck = 0;
+          ++s;
+        }
+        if (skip) continue;
+        int64_t last = rowA0 + (validB ? 255 : 127);
+        if (last > C - 1) last = C - 1;
+        tmax = diag ? (int)(last / BN) : ntiles - 1;
+        t = 0;
+        in_chunk = true;
+      }
+      if (t > tmax) {
+        in_chunk = false;
+        continue;
+      }
+      key0 = t * BN;
+      ++t;
+      actA = validA && (!diag || key0 <= rowA0 + 127);
+      actB = validB && (!diag || key0 <= rowA0 + 255);
+      if (!(actA || actB)) continue;
+      const bool tail = (int64_t)key0 + BN > C;
+      maskA = (diag && (int64_t)key0 + BN - 1 > rowA0) || tail;
+      maskB = (diag && (int64_t)key0 + BN - 1 > rowA0 + 128) || tail;
+      kv_row = base_row + key0;
+      return true;
+    }
+  }
+};
+
+template <int D>
+struct Smem {
+  static constexpr int QT = BM * D * 2;   // one Q tile
+  static constexpr int KT = BN * D * 2;   // one K or V tile (a ring stage)
+  static constexpr int PT = BM * BN * 2;  // one P tile
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_P = 2 * QT;
+  static constexpr int OFF_KV = OFF_P + 2 * PT;
+  static constexpr int OFF_BAR = OFF_KV + NSTAGE * KT;
+  static constexpr int NBAR = 2 * NSTAGE + 2 + 5 * 2;
+  static constexpr int BYTES = OFF_BAR + NBAR * 8 + 16;
+  static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Params p) {
+  using L = Smem<D>;
+  constexpr int NH = D / 64;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+
+  const uint32_t sQ0 = base + L::OFF_Q, sQ1 = sQ0 + L::QT;
+  const uint32_t sP0 = base + L::OFF_P, sP1 = sP0 + L::PT;
+  const uint32_t sKV = base + L::OFF_KV;
+  const uint32_t bar0 = base + L::OFF_BAR;
+  auto kv_full = [&](int i) { return bar0 + 8u * i; };
+  auto kv_empty = [&](int i) { return bar0 + 8u * (NSTAGE + i); };
+  const uint32_t q_full = bar0 + 8u * (2 * NSTAGE);
+  const uint32_t q_empty = q_full + 8u;
+  auto s_full = [&](int x) { return q_empty + 8u + 8u * x; };
+  auto s_free = [&](int x) { return q_empty + 24u + 8u * x; };
+  auto p_full = [&](int x) { return q_empty + 40u + 8u * x; };
+  auto o_done = [&](int x) { return q_empty + 56u + 8u * x; };
+  auto o_free = [&](int x) { return q_empty + 72u + 8u * x; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::OFF_BAR + L::NBAR * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::OFF_BAR + L::NBAR * 8 + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NSTAGE; ++i) {
+      mbar_init(kv_full(i), 1);
+      mbar_init(kv_empty(i), 1);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(s_full(x), 1);
+      mbar_init(s_free(x), 4);
+      mbar_init(p_full(x), 4);
+      mbar_init(o_done(x), 1);
+      mbar_init(o_free(x), 4);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const long long cap = p.wait_cap;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      int64_t pos = 0;
+      uint32_t qcnt = 0;
+      for (int64_t idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
+        const Item it = decode_item(p, idx);
+        if (qcnt > 0) mbar_wait(q_empty, (qcnt - 1) & 1, abort_flag, cap);
+        mbar_arrive_expect_tx(q_full, (uint32_t)((it.validA ? 1 : 0) + (it.validB ? 1 : 0)) * L::QT);
+        const int rowA = (int)((int64_t)it.r * 2 * p.C + (int64_t)it.c * p.C + it.rowA0);
+#pragma unroll
+        for (int hf = 0; hf < NH; ++hf) {
+          tma_load_3d(sQ0 + hf * HALF, &tmQ, q_full, hf * 64, it.h, rowA);
+          if (it.validB) tma_load_3d(sQ1 + hf * HALF, &tmQ, q_full, hf * 64, it.h, rowA + 128);
+        }
+        ++qcnt;
+        TileIter ti(p, it);
+        while (ti.next()) {
+#pragma unroll
+          for (int kv = 0; kv < 2; ++kv) {
+            const int st = (int)(pos % NSTAGE);
+            const uint32_t use = (uint32_t)(pos / NSTAGE);
+            mbar_wait(kv_empty(st), (use & 1) ^ 1, abort_flag, cap);
+            mbar_arrive_expect_tx(kv_full(st), L::KT);
+#pragma unroll
+            for (int hf = 0; hf < NH; ++hf)
+              tma_load_3d(sKV + st * L::KT + hf * HALF, kv ? (const void*)&tmV : (const void*)&tmK, kv_full(st),
+                          hf * 64, it.kvh, (int)ti.kv_row);
+            ++pos;
+          }
+        }
+      }
+      // Drain: every load issued must have landed before the CTA exits.
+      volatile int no_abort = 0;
+      for (int64_t i = (pos > NSTAGE ? pos - NSTAGE : 0); i < pos; ++i)
+        mbar_wait(kv_full((int)(i % NSTAGE)), (uint32_t)((i / NSTAGE) & 1), &no_abort, cap);
+      if (qcnt > 0) mbar_wait(q_full, (qcnt - 1) & 1, &no_abort, cap);
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
+      constexpr uint32_t idO = idesc_bf16_f32(BM, D, 0, 1);
+      const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
+      const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
+      const uint32_t sQ[2] = {sQ0, sQ1};
+      const uint32_t sP[2] = {sP0, sP1};
+      const std::integral_constant<int, 0> kA{};
+      const std::integral_constant<int, 1> kB{};
+      int64_t pos = 0;
+      uint32_t qcnt = 0;
+      uint32_t s_cnt[2] = {0, 0}, pv_cnt[2] = {0, 0}, epi_cnt[2] = {0, 0};
+
+      auto wait_full = [&](int64_t ps) {
+        mbar_wait(kv_full((int)(ps % NSTAGE)), (uint32_t)((ps / NSTAGE) & 1), abort_flag, cap);
+        tc_fence_after();
+      };
+      bool first_pv[2] = {true, true};
+      auto issue_S = [&](auto X, int64_t kpos) {
+        constexpr int x = decltype(X)::value;
+        if (s_cnt[x] > 0) {
+          mbar_wait(s_free(x), (s_cnt[x] - 1) & 1, abort_flag, cap);
+          tc_fence_after();
+        }
+        const uint32_t sk = sKV + (uint32_t)(kpos % NSTAGE) * L::KT;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
+          mma_bf16_ss(tS[x], desc_kmajor_sw128(sQ[x] + off), desc_kmajor_sw128(sk + off), idS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(s_full(x));
+        ++s_cnt[x];
+      };
+      auto issue_PV = [&](auto X, int64_t vpos) {
+        constexpr int x = decltype(X)::value;
+        mbar_wait(p_full(x), pv_cnt[x] & 1, abort_flag, cap);
+        tc_fence_after();
+        if (first_pv[x] && epi_cnt[x] > 0) {
+          mbar_wait(o_free(x), (epi_cnt[x] - 1) & 1, abort_flag, cap);
+          tc_fence_after();
+        }
+        const uint32_t sv = sKV + (uint32_t)(vpos % NSTAGE) * L::KT;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * HALF + (kk & 3) * 32;
+          mma_bf16_ss(tO[x], desc_kmajor_sw128(sP[x] + aoff), desc_mnmajor_sw128(sv + kk * 2048, HALF), idO,
+                      (kk > 0 || !first_pv[x]) ? 1u : 0u);
+        }
+        mma_commit(o_done(x));
+        ++pv_cnt[x];
+        first_pv[x] = false;
+      };
+
+      for (int64_t idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
+        const Item it = decode_item(p, idx);
+        mbar_wait(q_full, qcnt & 1, abort_flag, cap);
+        ++qcnt;
+        tc_fence_after();
+        first_pv[0] = first_pv[1] = true;
+        TileIter ti(p, it);
+        bool has = ti.next();
+        if (has) {
+          const int64_t kpos = pos++;
+          wait_full(kpos);
+          if (ti.actA) issue_S(kA, kpos);
+          if (ti.actB) issue_S(kB, kpos);
+          mma_commit(kv_empty((int)(kpos % NSTAGE)));
+        }
+        while (has) {
+          const bool curA = ti.actA, curB = ti.actB;
+          const int64_t vpos = pos++;
+          wait_full(vpos);
+          const bool has_next = ti.next();
+          int64_t kn = -1;
+          if (curA) issue_PV(kA, vpos);
+          if (has_next) {
+            kn = pos++;
+            wait_full(kn);
+            if (ti.actA) issue_S(kA, kn);
+          }
+          if (curB) issue_PV(kB, vpos);
+          mma_commit(kv_empty((int)(vpos % NSTAGE)));
+          if (has_next) {
+            if (ti.actB) issue_S(kB, kn);
+            mma_commit(kv_empty((int)(kn % NSTAGE)));
+          }
+          has = has_next;
+        }
+        mma_commit(q_empty);
+        if (!first_pv[0]) ++epi_cnt[0];
+        if (!first_pv[1]) ++epi_cnt[1];
+      }
+    }
+  } else {
+    // --------------------------------------------------- softmax groups
+    const int grp = (warp - 2) >> 2;  // 0: tile A, 1: tile B
+    const int wq = warp & 3;           // TMEM lane quarter this warp may access
+    const int row = wq * 32 + lane;    // row of the tile = TMEM lane
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + (uint32_t)(grp * 128) + lane_off;
+    const uint32_t tO = tmem + 256u + (uint32_t)(grp * D) + lane_off;
+    const uint32_t sPx = grp ? sP1 : sP0;
+    const float sl2 = p.scale_log2;
+    uint32_t s_cnt = 0, pv_cnt = 0;
+
+    for (int64_t idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
+      const Item it = decode_item(p, idx);
+      const bool valid = grp ? it.validB : it.validA;
+      if (!valid) continue;
+      const int64_t rin = it.rowA0 + grp * 128 + row;  // row within the chunk
+      float m = -CUDART_INF_F, l = 0.f;
+      int n_pv = 0;
+      TileIter ti(p, it);
+      while (ti.next()) {
+        if (!(grp ? ti.actB : ti.actA)) continue;
+        const bool msk = grp ? ti.maskB : ti.maskA;
+        mbar_wait(s_full(grp), s_cnt & 1, abort_flag, cap);
+        ++s_cnt;
+        tc_fence_after();
+        int64_t lim = 128;  // visible columns of this row in the tile
+        if (msk) {
+          lim = ti.C - ti.key0;
+          if (ti.diag) {
+            const int64_t dl = rin - ti.key0 + 1;
+            lim = dl < lim ? dl : lim;
+          }
+        }
+        // pass 1: row max over the tile, 64 columns per TMEM round trip
+        float mx = -CUDART_INF_F;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t sr[64];
+          tmem_ld32(tS + 64u * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          tmem_ld32(tS + 64u * h + 32u, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 64; ++j)
+            if (64 * h + j < lim) mx = fmaxf(mx, __uint_as_float(sr[j]));
+        }
+        const float mc = fmaxf(m, mx * sl2);
+        const bool need = mc > m + 8.0f;
+        float alpha = 1.f;
+        if (need) {
+          alpha = ex2_approx(m - mc);
+          m = mc;
+        }
+        const float mu = (m == -CUDART_INF_F) ? 0.f : m;
+        // The previous PV of this group is complete (it was issued before
+        // this S and tcgen05 work completes in order); the wait is cheap and
+        // makes the P buffer reuse explicit.
+        if (pv_cnt > 0) {
+          mbar_wait(o_done(grp), (pv_cnt - 1) & 1, abort_flag, cap);
+          tc_fence_after();
+        }
+        // pass 2: P = 2^(s*scale*log2e - m) as bf16 into the K-major,
+        // 128-byte-swizzled P tile (half h holds keys [64h, 64h+64)).
+        float rs = 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t sr[64];
+          tmem_ld32(tS + 64u * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          tmem_ld32(tS + 64u * h + 32u, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int j0 = 8 * c + 2 * u;
+              float e0 = ex2_approx(fmaf(__uint_as_float(sr[j0]), sl2, -mu));
+              float e1 = ex2_approx(fmaf(__uint_as_float(sr[j0 + 1]), sl2, -mu));
+              if (64 * h + j0 >= lim) e0 = 0.f;
+              if (64 * h + j0 + 1 >= lim) e1 = 0.f;
+              rs += e0 + e1;
+              pk[u] = pack_bf16x2(e0, e1);
+            }
+            const uint32_t addr = sPx + h * HALF + row * 128 + ((((uint32_t)c) ^ ((uint32_t)row & 7u)) << 4);
+            st_shared_v4(addr, pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free(grp));
+        l = l * alpha + rs;
+        if (n_pv > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32u * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+            tmem_st32(tO + 32u * c, o);
+          }
+          tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full(grp));
+        ++pv_cnt;
+        ++n_pv;
+      }
+
+      // ---------------------------------------------------------- epilogue
+      // O = acc / l and LSE = (m + log2 l) ln 2, merged into the running
+      // state when accumulating; written 32 columns at a time.
+      const float LN2 = 0.6931471805599453f;
+      float lse_new = -CUDART_INF_F;
+      float inv = 0.f;
+      if (l > 0.f) {
+        lse_new = (m + log2f(l)) * LN2;
+        inv = 1.f / l;
+      }
+      const bool row_ok = rin < p.C;
+      const int64_t lrow = (int64_t)it.r * 2 * p.C + (int64_t)it.c * p.C + rin;
+      const int64_t rh = lrow * p.Hq + it.h;
+      float wa = 0.f, wb = inv, L = lse_new;
+      float4* oacc = (p.o_acc && row_ok) ? reinterpret_cast<float4*>(p.o_acc + rh * D) : nullptr;
+      if (p.accumulate && row_ok) {
+        const float lo = p.lse[rh];
+        const float mm = fmaxf(lo, lse_new);
+        if (mm == -CUDART_INF_F) {
+          wb = 0.f;
+          L = -CUDART_INF_F;
+        } else {
+          const float ea = expf(lo - mm), eb = expf(lse_new - mm);
+          const float sum = ea + eb;
+          L = mm + logf(sum);
+          wa = ea / sum;
+          wb = inv * (eb / sum);
+        }
+      }
+      if (row_ok) p.lse[rh] = L;
+      if (n_pv > 0) {
+        mbar_wait(o_done(grp), (pv_cnt - 1) & 1, abort_flag, cap);
+        tc_fence_after();
+      }
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t acc[32];
+        if (n_pv > 0) {
+          tmem_ld32(tO + 32u * c, acc);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[j] = 0u;
+        }
+        if (row_ok) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            float4 v;
+            v.x = __uint_as_float(acc[j + 0]) * wb;
+            v.y = __uint_as_float(acc[j + 1]) * wb;
+            v.z = __uint_as_float(acc[j + 2]) * wb;
+            v.w = __uint_as_float(acc[j + 3]) * wb;
+            const int q4 = (32 * c + j) / 4;
+            if (p.accumulate) {
+              const float4 old = oacc[q4];
+              v.x += wa * old.x;
+              v.y += wa * old.y;
+              v.z += wa * old.z;
+              v.w += wa * old.w;
+            }
+            if (oacc) oacc[q4] = v;
+            if (p.finalize) {
+              uint2 bb;
+              bb.x = pack_bf16x2(v.x, v.y);
+              bb.y = pack_bf16x2(v.z, v.w);
+              reinterpret_cast<uint2*>(p.o_out + rh * D)[q4] = bb;
+            }
+          }
+        }
+      }
+      if (n_pv > 0) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(o_free(grp));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fwd
+}  // namespace mmsp

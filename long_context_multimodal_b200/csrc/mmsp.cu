@@ -1,0 +1,332 @@
+// mmsp.cu -- the C ABI of libmmsp.so (declared in include/mmsp.h): host-side
+// validation, TMA descriptor encoding and stream-ordered launches of the
+// sm_100a kernels. One translation unit so that every kernel shares the
+// device-side timeout flag. The library allocates no device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "mmsp.h"
+#include "ptx.cuh"
+#include "shard.cuh"
+#include "merge.cuh"
+#include "attn_fwd.cuh"
+#include "attn_bwd.cuh"
+
+using namespace mmsp;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int ok() {
+  g_err[0] = 0;
+  return MMSP_OK;
+}
+
+#define MMSP_CUDA(call)                                                                        \
+  do {                                                                                         \
+    cudaError_t e_ = (call);                                                                   \
+    if (e_ != cudaSuccess) return fail(MMSP_ECUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  int sms = 0;
+  bool fwd_attr[2] = {false, false};
+  bool bwd_attr[2] = {false, false};
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+int current_device(int* dev) {
+  MMSP_CUDA(cudaGetDevice(dev));
+  if (*dev < 0 || *dev >= kMaxDevices) return fail(MMSP_EUNSUPPORTED, "device index %d out of range", *dev);
+  return MMSP_OK;
+}
+
+int device_sms(int dev, int* sms) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_dev[dev].sms == 0) {
+    int v = 0;
+    MMSP_CUDA(cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev));
+    g_dev[dev].sms = v;
+  }
+  *sms = g_dev[dev].sms;
+  return MMSP_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int get_encode() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode) return MMSP_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess || fn == nullptr || q != cudaDriverEntryPointSuccess)
+    return fail(MMSP_ECUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return MMSP_OK;
+}
+
+// [rows][H][D] bf16 viewed as 3-D (d, head, row); boxes of 64 d x 1 head x
+// 128 rows with 128-byte swizzle (one 128-byte line per row and box).
+int tmap_rows_heads(CUtensorMap* m, const void* ptr, int64_t rows, int H, int D) {
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MMSP_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MMSP_OK;
+}
+
+// Caps for the device-side bounded waits, in SM clock cycles (about 2 s).
+constexpr long long kWaitCapCycles = 1LL << 32;
+
+int check_common(int64_t N, int32_t P) {
+  if (N < 0) return fail(MMSP_EINVAL, "N must be >= 0 (got %lld)", (long long)N);
+  if (P < 1) return fail(MMSP_EINVAL, "P must be >= 1 (got %d)", P);
+  if (N >= (int64_t(1) << 31)) return fail(MMSP_EINVAL, "N must be < 2^31 (got %lld)", (long long)N);
+  if (N % (2 * (int64_t)P) != 0) return fail(MMSP_EINVAL, "N (%lld) must be divisible by 2P (%d)", (long long)N, 2 * P);
+  return MMSP_OK;
+}
+
+int check_heads(int32_t Hq, int32_t Hkv, int32_t d) {
+  if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return fail(MMSP_EINVAL, "need Hq %% Hkv == 0, Hq, Hkv >= 1 (Hq=%d Hkv=%d)", Hq, Hkv);
+  if (d != 64 && d != 128) return fail(MMSP_EINVAL, "head dim d must be 64 or 128 (got %d)", d);
+  return MMSP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mmsp_last_error(void) { return g_err; }
+
+const char* mmsp_version(void) { return "mmsp 0.1 (sm_100a)"; }
+
+int mmsp_shard(const int32_t* seg_len, const uint8_t* seg_kind, int32_t n_seg, int64_t N, int32_t P,
+               int32_t* local2global, int32_t* global2local, uint8_t* modality_local, int32_t* segid_local,
+               int32_t* rank_counts, const void* src, void* dst, int64_t row_bytes, int32_t inverse, void* stream) {
+  int rc = check_common(N, P);
+  if (rc) return rc;
+  const bool need_seg = modality_local || segid_local || rank_counts;
+  if (need_seg) {
+    if (!seg_len || !seg_kind) return fail(MMSP_EINVAL, "segment table required for modality/segid/rank_counts");
+    if (n_seg < 1 || n_seg > MMSP_MAX_SEGMENTS)
+      return fail(MMSP_EINVAL, "n_seg must be in [1, %d] (got %d)", MMSP_MAX_SEGMENTS, n_seg);
+  }
+  if ((src == nullptr) != (dst == nullptr)) return fail(MMSP_EINVAL, "src and dst must both be set or both NULL");
+  if (src) {
+    if (row_bytes <= 0 || row_bytes % 16) return fail(MMSP_EINVAL, "row_bytes must be a positive multiple of 16");
+    if (!aligned16(src) || !aligned16(dst)) return fail(MMSP_EINVAL, "src/dst must be 16-byte aligned");
+    const char* s = static_cast<const char*>(src);
+    const char* e = static_cast<const char*>(dst);
+    const int64_t bytes = N * row_bytes;
+    if (s < e + bytes && e < s + bytes) return fail(MMSP_EINVAL, "src and dst overlap");
+  }
+  static SegTable tab;  // host staging; copied into the launch parameters
+  static std::mutex tab_mu;
+  std::lock_guard<std::mutex> lk(tab_mu);
+  if (need_seg) {
+    int64_t acc = 0;
+    tab.n = n_seg;
+    for (int i = 0; i < n_seg; ++i) {
+      if (seg_len[i] < 1) return fail(MMSP_EINVAL, "segment %d has length %d < 1", i, seg_len[i]);
+      if (seg_kind[i] > 1) return fail(MMSP_EINVAL, "segment %d has kind %d (0 text, 1 visual)", i, seg_kind[i]);
+      tab.start[i] = (int32_t)acc;
+      tab.kind[i] = seg_kind[i];
+      acc += seg_len[i];
+      if (acc > N) break;
+    }
+    if (acc != N) return fail(MMSP_EINVAL, "segment lengths sum to %lld, expected N=%lld", (long long)acc, (long long)N);
+    tab.start[n_seg] = (int32_t)N;
+  } else {
+    tab.n = 0;
+    tab.start[0] = 0;
+  }
+  if (N == 0) return ok();
+  int dev, sms;
+  if ((rc = current_device(&dev)) || (rc = device_sms(dev, &sms))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (local2global || global2local || modality_local || segid_local) {
+    int64_t blocks = (N + 255) / 256;
+    if (blocks > 8LL * sms) blocks = 8LL * sms;
+    shard_maps_kernel<<<(unsigned)blocks, 256, 0, st>>>(tab, (int32_t)N, P, local2global, global2local,
+                                                         modality_local, segid_local);
+    MMSP_CUDA(cudaGetLastError());
+  }
+  if (rank_counts) {
+    shard_counts_kernel<<<1, 256, 0, st>>>(tab, (int32_t)N, P, rank_counts);
+    MMSP_CUDA(cudaGetLastError());
+  }
+  if (src) {
+    int64_t blocks = (N + 7) / 8;  // 8 warps (rows) per block
+    if (blocks > 16LL * sms) blocks = 16LL * sms;
+    shard_rows_kernel<<<(unsigned)blocks, 256, 0, st>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst),
+                                                         (int32_t)N, P, row_bytes / 16, inverse ? 1 : 0);
+    MMSP_CUDA(cudaGetLastError());
+  }
+  return ok();
+}
+
+int mmsp_lse_merge(const float* o_a, const float* lse_a, const float* o_b, const float* lse_b, float* o_out,
+                   float* lse_out, int64_t rows, int32_t H, int32_t d, void* stream) {
+  if (rows < 0 || H < 1) return fail(MMSP_EINVAL, "rows must be >= 0 and H >= 1");
+  if (!(d == 4 || d == 8 || d == 16 || d == 32 || d == 64 || d == 128))
+    return fail(MMSP_EINVAL, "d must be one of 4, 8, 16, 32, 64, 128 (got %d)", d);
+  if (!o_a || !lse_a || !o_b || !lse_b || !o_out || !lse_out) return fail(MMSP_EINVAL, "NULL pointer");
+  if (!aligned16(o_a) || !aligned16(o_b) || !aligned16(o_out))
+    return fail(MMSP_EINVAL, "o_a, o_b, o_out must be 16-byte aligned");
+  if (((uintptr_t)lse_a | (uintptr_t)lse_b | (uintptr_t)lse_out) & 3u) return fail(MMSP_EINVAL, "lse pointers must be 4-byte aligned");
+  const int64_t total = rows * H;
+  if (total == 0) return ok();
+  int dev, sms, rc;
+  if ((rc = current_device(&dev)) || (rc = device_sms(dev, &sms))) return rc;
+  int64_t warps = (total + 31) / 32;
+  int64_t blocks = (warps + 7) / 8;
+  if (blocks > 8LL * sms) blocks = 8LL * sms;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+#define MMSP_MERGE(DD) \
+  case DD:             \
+    lse_merge_kernel<DD><<<(unsigned)blocks, 256, 0, st>>>(o_a, lse_a, o_b, lse_b, o_out, lse_out, total); break;
+  switch (d) { MMSP_MERGE(4) MMSP_MERGE(8) MMSP_MERGE(16) MMSP_MERGE(32) MMSP_MERGE(64) MMSP_MERGE(128) }
+#undef MMSP_MERGE
+  MMSP_CUDA(cudaGetLastError());
+  return ok();
+}
+
+int mmsp_attn_fwd(const void* q, const void* k, const void* v, int64_t N, int32_t P, int32_t Hq, int32_t Hkv,
+                  int32_t d, float scale, int32_t causal, int32_t step_begin, int32_t step_end, float* o_acc,
+                  float* lse, void* o_out, uint32_t flags, void* stream) {
+  int rc = check_common(N, P);
+  if (rc) return rc;
+  if ((rc = check_heads(Hq, Hkv, d))) return rc;
+  if (flags & ~(MMSP_ACCUMULATE | MMSP_FINALIZE)) return fail(MMSP_EINVAL, "unknown flags 0x%x", flags);
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(MMSP_EINVAL, "scale must be finite and > 0");
+  if (causal != 0 && causal != 1) return fail(MMSP_EINVAL, "causal must be 0 or 1");
+  if (step_begin < 0 || step_end < step_begin || step_end > P)
+    return fail(MMSP_EINVAL, "need 0 <= step_begin <= step_end <= P (got %d, %d, P=%d)", step_begin, step_end, P);
+  if (!q || !k || !v || !lse) return fail(MMSP_EINVAL, "q, k, v and lse must be non-NULL");
+  if ((flags & MMSP_ACCUMULATE) && !o_acc) return fail(MMSP_EINVAL, "MMSP_ACCUMULATE needs o_acc");
+  if ((flags & MMSP_FINALIZE) && !o_out) return fail(MMSP_EINVAL, "MMSP_FINALIZE needs o_out");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(lse) || (o_acc && !aligned16(o_acc)) ||
+      (o_out && !aligned16(o_out)))
+    return fail(MMSP_EINVAL, "all tensors must be 16-byte aligned");
+  if (N == 0) return ok();
+  int dev, sms;
+  if ((rc = current_device(&dev)) || (rc = device_sms(dev, &sms)) || (rc = get_encode())) return rc;
+  CUtensorMap tq, tk, tv;
+  if ((rc = tmap_rows_heads(&tq, q, N, Hq, d)) || (rc = tmap_rows_heads(&tk, k, N, Hkv, d)) ||
+      (rc = tmap_rows_heads(&tv, v, N, Hkv, d)))
+    return rc;
+  fwd::Params p;
+  p.P = P;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.C = N / (2 * (int64_t)P);
+  p.nblk = (int32_t)((p.C + 255) / 256);
+  p.causal = causal;
+  p.step_begin = step_begin;
+  p.step_end = step_end;
+  p.accumulate = (flags & MMSP_ACCUMULATE) ? 1 : 0;
+  p.finalize = (flags & MMSP_FINALIZE) ? 1 : 0;
+  p.n_items = 2LL * P * p.nblk * Hq;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o_acc = o_acc;
+  p.lse = lse;
+  p.o_out = static_cast<__nv_bfloat16*>(o_out);
+  p.wait_cap = kWaitCapCycles;
+  const int64_t grid = p.n_items < sms ? p.n_items : sms;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int di = d == 128 ? 1 : 0;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_dev[dev].fwd_attr[di]) {
+      if (d == 128)
+        MMSP_CUDA(cudaFuncSetAttribute(fwd::attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       fwd::Smem<128>::ALLOC));
+      else
+        MMSP_CUDA(cudaFuncSetAttribute(fwd::attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       fwd::Smem<64>::ALLOC));
+      g_dev[dev].fwd_attr[di] = true;
+    }
+  }
+  if (d == 128)
+    fwd::attn_fwd_kernel<128><<<(unsigned)grid, fwd::kThreads, fwd::Smem<128>::ALLOC, st>>>(tq, tk, tv, p);
+  else
+    fwd::attn_fwd_kernel<64><<<(unsigned)grid, fwd::kThreads, fwd::Smem<64>::ALLOC, st>>>(tq, tk, tv, p);
+  MMSP_CUDA(cudaGetLastError());
+  return ok();
+}
+
+int mmsp_device_status(void* stream) {
+  MMSP_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  MMSP_CUDA(cudaGetLastError());
+  int flag = 0;
+  MMSP_CUDA(cudaMemcpyFromSymbol(&flag, g_timeout_flag, sizeof(int)));
+  if (flag) {
+    const int zero = 0;
+    MMSP_CUDA(cudaMemcpyToSymbol(g_timeout_flag, &zero, sizeof(int)));
+    return fail(MMSP_ETIMEOUT, "a bounded device-side wait gave up");
+  }
+  return ok();
+}
+
+}  // extern "C"
+
+namespace {
+__global__ void selftest_wait_kernel(long long max_cycles) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_word;
+  if (threadIdx.x == 0) {
+    mmsp::mbar_init(mmsp::smem_u32(&bar), 1);
+    abort_word = 0;
+    mmsp::fence_barrier_init();
+  }
+  __syncthreads();
+  // Nobody arrives: the wait must give up and record the timeout.
+  mmsp::mbar_wait(mmsp::smem_u32(&bar), 0, &abort_word, max_cycles);
+}
+}  // namespace
+
+extern "C" int mmsp_selftest_bounded_wait(int64_t max_cycles, void* stream) {
+  if (max_cycles < 1 || max_cycles > (int64_t(1) << 31))
+    return fail(MMSP_EINVAL, "max_cycles must be in [1, 2^31]");
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((long long)max_cycles);
+  MMSP_CUDA(cudaGetLastError());
+  return ok();
+}
+
+extern "C" size_t mmsp_bwd_workspace_bytes(int64_t N, int32_t P, int32_t Hq, int32_t d) {
+  (void)N; (void)P; (void)Hq; (void)d;
+  return 0;
+}
+
+extern "C" int mmsp_attn_bwd(const void*, const void*, const void*, const void*, const void*, const float*, int64_t,
+                             int32_t, int32_t, int32_t, int32_t, float, int32_t, void*, void*, void*, float*, void*,
+                             size_t, void*) {
+  return fail(MMSP_EUNSUPPORTED, "backward not built yet");
+}

@@ -22,15 +22,22 @@ above), with P_ij = exp(s_ij - LSE_i) and D_i = sum_d dO_i * O_i:
 
 Inputs are numpy arrays (any float dtype; converted to fp64) of shape
 [N, H, d]. Rows are processed in blocks only to bound memory; every block is
-the plain formula.
+the plain formula, evaluated with fp64 torch CPU ops (matmul, exp, log,
+max, sum) so that large sampled checks use every host core.
 """
 from __future__ import annotations
 
 import math
 
 import numpy as np
+import torch
 
 NEG_INF = -np.inf
+
+
+def _t(x):
+    """fp64 CPU torch view of a numpy array (no copy when already fp64)."""
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64))
 
 
 def kv_head(h: int, hq: int, hkv: int) -> int:
@@ -46,22 +53,23 @@ def _f64(x):
 
 def _rows_forward(qr, rows, K, V, scale):
     """O and LSE for query vectors qr [R,d] at global positions rows [R]
-    against keys K[:i+1], V[:i+1] (one head)."""
+    against keys K[:i+1], V[:i+1] (one head). Plain formula in fp64 torch
+    CPU ops (multi-threaded; same arithmetic as numpy)."""
     R = len(rows)
     d = V.shape[1]
-    O = np.zeros((R, d))
-    L = np.full(R, NEG_INF)
     if R == 0:
-        return O, L
-    jmax = int(rows.max()) + 1
-    s = (qr @ K[:jmax].T) * scale                      # [R, jmax]
-    visible = np.arange(jmax)[None, :] <= rows[:, None]
-    s = np.where(visible, s, NEG_INF)
-    m = s.max(axis=1)
-    lse = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
-    p = np.exp(s - lse[:, None])                        # 0 where masked
-    O = p @ V[:jmax]
-    return O, lse
+        return np.zeros((R, d)), np.full(R, NEG_INF)
+    jmax = int(np.max(rows)) + 1
+    qr, K, V = _t(qr), _t(K[:jmax]), _t(V[:jmax])
+    rows_t = torch.as_tensor(np.asarray(rows, np.int64))
+    s = (qr @ K.T) * scale                                       # [R, jmax]
+    visible = torch.arange(jmax)[None, :] <= rows_t[:, None]
+    s = s.masked_fill(~visible, NEG_INF)
+    m = s.max(dim=1).values
+    lse = m + torch.log(torch.exp(s - m[:, None]).sum(dim=1))
+    p = torch.exp(s - lse[:, None])                              # 0 where masked
+    O = p @ V
+    return O.numpy(), lse.numpy()
 
 
 def causal_attention(q, k, v, scale=None, block: int = 512):
@@ -83,42 +91,55 @@ def causal_attention(q, k, v, scale=None, block: int = 512):
     return O, LSE
 
 
-def attention_rows(q, k, v, rows, scale=None, block: int = 64):
-    """Forward for selected global rows only. Returns (O [R,Hq,d], LSE [R,Hq])."""
-    q, k, v = _f64(q), _f64(k), _f64(v)
+def attention_rows(q_rows, k, v, rows, scale=None, block: int = 64):
+    """Forward for selected global rows only.
+
+    q_rows [R,Hq,d] holds the query vectors of global positions `rows` (the
+    caller gathers them, so the whole Q need not be held in fp64); k, v are
+    the whole [N,Hkv,d] tensors, converted to fp64 one kv head at a time.
+    Returns (O [R,Hq,d], LSE [R,Hq]).
+    """
+    q_rows = _f64(q_rows)
     rows = np.asarray(rows, np.int64)
-    N, hq, d = q.shape
+    R, hq, d = q_rows.shape
     hkv = k.shape[1]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    O = np.zeros((len(rows), hq, d))
-    LSE = np.zeros((len(rows), hq))
-    for h in range(hq):
-        kh = kv_head(h, hq, hkv)
-        for b0 in range(0, len(rows), block):
-            sel = np.arange(b0, min(len(rows), b0 + block))
-            o, l = _rows_forward(q[rows[sel], h], rows[sel], k[:, kh], v[:, kh], scale)
-            O[sel, h] = o
-            LSE[sel, h] = l
+    jmax = int(rows.max()) + 1 if R else 0
+    O = np.zeros((R, hq, d))
+    LSE = np.zeros((R, hq))
+    for kh in range(hkv):
+        K = _f64(k[:jmax, kh])
+        V = _f64(v[:jmax, kh])
+        for h in range(hq):
+            if kv_head(h, hq, hkv) != kh:
+                continue
+            for b0 in range(0, R, block):
+                sel = np.arange(b0, min(R, b0 + block))
+                o, l = _rows_forward(q_rows[sel, h], rows[sel], K, V, scale)
+                O[sel, h] = o
+                LSE[sel, h] = l
     return O, LSE
 
 
 def _rows_backward(qr, dor, rows, K, V, scale):
     """For one head and query rows: (O, LSE, D, dQ rows, P, dS) restricted to
-    keys [0, max(rows)]; P and dS are [R, jmax]."""
-    jmax = int(rows.max()) + 1
-    s = (qr @ K[:jmax].T) * scale
-    visible = np.arange(jmax)[None, :] <= rows[:, None]
-    s = np.where(visible, s, NEG_INF)
-    m = s.max(axis=1)
-    lse = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
-    p = np.exp(s - lse[:, None])
-    o = p @ V[:jmax]
-    D = (dor * o).sum(axis=1)
-    dp = dor @ V[:jmax].T
+    keys [0, max(rows)]; P and dS are [R, jmax]. fp64 torch CPU ops."""
+    jmax = int(np.max(rows)) + 1
+    qr, dor, K, V = _t(qr), _t(dor), _t(K[:jmax]), _t(V[:jmax])
+    rows_t = torch.as_tensor(np.asarray(rows, np.int64))
+    s = (qr @ K.T) * scale
+    visible = torch.arange(jmax)[None, :] <= rows_t[:, None]
+    s = s.masked_fill(~visible, NEG_INF)
+    m = s.max(dim=1).values
+    lse = m + torch.log(torch.exp(s - m[:, None]).sum(dim=1))
+    p = torch.exp(s - lse[:, None])
+    o = p @ V
+    D = (dor * o).sum(dim=1)
+    dp = dor @ V.T
     ds = p * (dp - D[:, None])
-    dq = scale * (ds @ K[:jmax])
-    return o, lse, D, dq, p, ds
+    dq = scale * (ds @ K)
+    return o.numpy(), lse.numpy(), D.numpy(), dq.numpy(), p.numpy(), ds.numpy()
 
 
 def causal_attention_bwd(q, k, v, do, scale=None, block: int = 512):
@@ -153,27 +174,31 @@ def causal_attention_bwd(q, k, v, do, scale=None, block: int = 512):
     return {"O": O, "LSE": LSE, "D": Dm, "dQ": dQ, "dK": dK, "dV": dV}
 
 
-def attention_bwd_rows(q, k, v, do, rows, scale=None, block: int = 64):
-    """dQ (and O, LSE) for selected global rows: row i needs only keys <= i."""
-    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+def attention_bwd_rows(q_rows, k, v, do_rows, rows, scale=None, block: int = 64):
+    """dQ (and O, LSE) for selected global rows: row i needs only keys <= i.
+    q_rows and do_rows [R,Hq,d] are the caller-gathered rows at `rows`."""
+    q_rows, do_rows = _f64(q_rows), _f64(do_rows)
     rows = np.asarray(rows, np.int64)
-    N, hq, d = q.shape
+    R, hq, d = q_rows.shape
     hkv = k.shape[1]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    R = len(rows)
+    jmax = int(rows.max()) + 1 if R else 0
     dQ = np.zeros((R, hq, d))
     O = np.zeros((R, hq, d))
     LSE = np.zeros((R, hq))
-    for h in range(hq):
-        kh = kv_head(h, hq, hkv)
-        for b0 in range(0, R, block):
-            sel = np.arange(b0, min(R, b0 + block))
-            o, lse, _, dq, _, _ = _rows_backward(q[rows[sel], h], do[rows[sel], h], rows[sel],
-                                                 k[:, kh], v[:, kh], scale)
-            dQ[sel, h] = dq
-            O[sel, h] = o
-            LSE[sel, h] = lse
+    for kh in range(hkv):
+        K = _f64(k[:jmax, kh])
+        V = _f64(v[:jmax, kh])
+        for h in range(hq):
+            if kv_head(h, hq, hkv) != kh:
+                continue
+            for b0 in range(0, R, block):
+                sel = np.arange(b0, min(R, b0 + block))
+                o, lse, _, dq, _, _ = _rows_backward(q_rows[sel, h], do_rows[sel, h], rows[sel], K, V, scale)
+                dQ[sel, h] = dq
+                O[sel, h] = o
+                LSE[sel, h] = lse
     return {"O": O, "LSE": LSE, "dQ": dQ}
 
 

@@ -110,3 +110,35 @@ def ring_attention(q, k, v, P: int, scale=None):
     Og = sharder.permute_rows(O.reshape(N, hq, d), l2g, inverse=True)
     Lg = sharder.permute_rows(L.reshape(N, hq), l2g, inverse=True)
     return Og, Lg, pairs
+
+
+def ring_step_partials(q, k, v, P: int, step: int, scale=None):
+    """Partial (O, LSE) of every virtual rank at one ring step, in rank-local
+    order [N, Hq, d] / [N, Hq]: rank r's queries against the K/V block it
+    holds after `step` receives from its previous ring rank."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    N, hq, d = q.shape
+    hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    maps = sharder.shard_maps([N], [0], N, P)
+    l2g = maps["local2global"]
+    C2 = N // P
+    ql = sharder.permute_rows(q, l2g)
+    kl = sharder.permute_rows(k, l2g)
+    vl = sharder.permute_rows(v, l2g)
+    pos = l2g.astype(np.int64)
+    cur = [(kl[r * C2:(r + 1) * C2], vl[r * C2:(r + 1) * C2], pos[r * C2:(r + 1) * C2]) for r in range(P)]
+    for _ in range(step):
+        cur = [cur[(r - 1) % P] for r in range(P)]
+    O = np.zeros((N, hq, d))
+    L = np.full((N, hq), NEG_INF)
+    for r in range(P):
+        kb, vb, kpos = cur[r]
+        sl = slice(r * C2, (r + 1) * C2)
+        for h in range(hq):
+            kh = (h * hkv) // hq
+            O[sl, h], L[sl, h] = block_attention(ql[sl, h], pos[sl], kb[:, kh], vb[:, kh], kpos, scale)
+    return O, L

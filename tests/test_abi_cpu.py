@@ -1,0 +1,94 @@
+"""The C-ABI library loads and exports every symbol include/mmsp.h declares;
+host-side validation rejects bad arguments before any launch (CPU only: no
+compute call reaches the GPU)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    text = open(os.path.join(ROOT, "include", "mmsp.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mmsp_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    import long_context_multimodal_b200 as m
+
+    names = _header_functions()
+    assert "mmsp_attn_fwd" in names and "mmsp_shard" in names and len(names) >= 9
+    lib = ctypes.CDLL(m.lib_path())
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(m.exported_symbols()) == set(names)
+    assert "sm_100a" in m.mmsp_version()
+
+
+def _einval(fn, *a, **k):
+    import long_context_multimodal_b200 as m
+
+    with pytest.raises(m.MmspError) as e:
+        fn(*a, **k)
+    assert e.value.status == 1, str(e.value)
+    return str(e.value)
+
+
+def test_attn_fwd_rejects_bad_arguments():
+    import long_context_multimodal_b200 as m
+
+    F = m.mmsp_attn_fwd
+    p = 1 << 20  # a 16-byte-aligned stand-in pointer; nothing is launched
+    ok = dict(q=p, k=p, v=p, N=4096, P=4, Hq=4, Hkv=4, d=64, scale=0.125, causal=1, step_begin=0, step_end=4,
+              o_acc=p, lse=p, o_out=p, flags=m.MMSP_FINALIZE)
+    for bad in [dict(N=4095), dict(N=4100, P=4), dict(P=0), dict(N=-2), dict(Hq=6, Hkv=4), dict(d=96),
+                dict(d=256), dict(step_begin=3, step_end=2), dict(step_end=5), dict(q=p + 8), dict(lse=None),
+                dict(scale=0.0), dict(scale=float("nan")), dict(causal=2), dict(flags=8),
+                dict(flags=m.MMSP_ACCUMULATE, o_acc=None), dict(o_out=None), dict(N=1 << 31, P=1)]:
+        args = dict(ok, **bad)
+        _einval(F, **args)
+
+
+def test_shard_rejects_bad_arguments():
+    import long_context_multimodal_b200 as m
+
+    p = 1 << 20
+    _einval(m.mmsp_shard, None, None, 10, 3)                                   # N % 2P
+    _einval(m.mmsp_shard, [5, 4], [0, 1], 8, 2, local2global=p, modality_local=p)  # sum != N
+    _einval(m.mmsp_shard, [8], [2], 8, 2, modality_local=p)                   # bad kind
+    _einval(m.mmsp_shard, [0, 8], [0, 0], 8, 2, segid_local=p)               # empty segment
+    _einval(m.mmsp_shard, None, None, 8, 2, modality_local=p)                 # table missing
+    _einval(m.mmsp_shard, np.ones(4097, np.int32), np.zeros(4097, np.uint8), 4097 * 2, 1,
+            rank_counts=p)                                                     # over capacity
+    _einval(m.mmsp_shard, None, None, 8, 2, src=p, dst=None)                  # half a permute
+    _einval(m.mmsp_shard, None, None, 8, 2, src=p, dst=p + 4096, row_bytes=24)  # row_bytes % 16
+    _einval(m.mmsp_shard, None, None, 8, 2, src=p, dst=p + 64, row_bytes=16)  # overlap
+
+
+def test_merge_and_bwd_reject_bad_arguments():
+    import long_context_multimodal_b200 as m
+
+    p = 1 << 20
+    _einval(m.mmsp_lse_merge, p, p, p, p, p, p, 10, 2, 96)
+    _einval(m.mmsp_lse_merge, p + 4, p, p, p, p, p, 10, 2, 64)
+    _einval(m.mmsp_lse_merge, p, p, p, p, p, p, -1, 2, 64)
+    _einval(m.mmsp_selftest_bounded_wait, 0)
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    """The binding has no fallback: a missing .so is an ImportError."""
+    import importlib.util
+    import shutil
+
+    pkg = os.path.join(ROOT, "long_context_multimodal_b200")
+    dst = tmp_path / "pkgcopy"
+    shutil.copytree(pkg, dst, ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    spec = importlib.util.spec_from_file_location("pkgcopy", dst / "__init__.py",
+                                                  submodule_search_locations=[str(dst)])
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError):
+        spec.loader.exec_module(mod)

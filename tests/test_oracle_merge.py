@@ -93,3 +93,36 @@ def test_ring_steps_have_two_full_blocks_after_step_zero(N, P):
     if P > 1:
         assert np.all(pairs[:, 1:] == 2 * C * C)
     assert np.all(pairs.sum(axis=1) == C * (2 * P * C + 1))
+
+
+def test_ring_step_partials_merge_to_full_and_follow_ring_order():
+    """The per-step partials merged over all steps equal the definition, and
+    step s gives rank r exactly the keys of rank (r - s) mod P."""
+    N, P = 48, 4
+    C = N // (2 * P)
+    rng = np.random.default_rng(9)
+    q = rng.standard_normal((N, 2, 8))
+    k = rng.standard_normal((N, 1, 8))
+    v = rng.standard_normal((N, 1, 8))
+    Ol, Ll = None, None
+    for s in range(P):
+        o, l = M.ring_step_partials(q, k, v, P, s)
+        if Ol is None:
+            Ol, Ll = o, l
+        else:
+            Ol, Ll = M.lse_merge(Ol, Ll, o, l)
+        # rank 1 at step 1 holds rank 0's K/V (chunks 0 and 2P-1); its chunk-0
+        # queries (global chunk 1) see all of chunk 0 and nothing of chunk 2P-1
+        if s == 1:
+            r = 1
+            rows = slice(r * 2 * C, r * 2 * C + C)
+            g0 = np.arange(0, C)
+            ref_o, ref_l = M.block_attention(q[C:2 * C, 0], np.arange(C, 2 * C), k[g0, 0], v[g0, 0], g0,
+                                             1 / np.sqrt(8))
+            np.testing.assert_allclose(o[rows, 0], ref_o, atol=1e-12)
+            np.testing.assert_allclose(l[rows, 0], ref_l, atol=1e-12)
+    from oracle import sharder
+    l2g = sharder.shard_maps([N], [0], N, P)["local2global"]
+    Og = sharder.permute_rows(Ol, l2g, inverse=True)
+    Or, Lr = A.causal_attention(q, k, v)
+    np.testing.assert_allclose(Og, Or, atol=1e-12)
