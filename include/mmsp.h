@@ -79,8 +79,9 @@ typedef enum {
  *   src, dst           DEVICE row buffers or both NULL. With inverse == 0:
  *                      dst[l] = src[local2global(l)] (global -> rank-local);
  *                      with inverse != 0: dst[local2global(l)] = src[l].
- *                      Rows are row_bytes long; src, dst and row_bytes must be
- *                      multiples of 16 bytes; src and dst must not overlap.
+ *                      Rows are row_bytes long, a multiple of 4 bytes; src and
+ *                      dst 16-byte aligned when row_bytes % 16 == 0 (16-byte
+ *                      vector path), else 4-byte aligned; no overlap.
  * Bit-exact: pure integer / byte work.
  */
 int mmsp_shard(const int32_t* seg_len, const uint8_t* seg_kind, int32_t n_seg,

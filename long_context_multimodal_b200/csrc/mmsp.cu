@@ -139,8 +139,10 @@ int mmsp_shard(const int32_t* seg_len, const uint8_t* seg_kind, int32_t n_seg, i
   }
   if ((src == nullptr) != (dst == nullptr)) return fail(MMSP_EINVAL, "src and dst must both be set or both NULL");
   if (src) {
-    if (row_bytes <= 0 || row_bytes % 16) return fail(MMSP_EINVAL, "row_bytes must be a positive multiple of 16");
-    if (!aligned16(src) || !aligned16(dst)) return fail(MMSP_EINVAL, "src/dst must be 16-byte aligned");
+    if (row_bytes <= 0 || row_bytes % 4) return fail(MMSP_EINVAL, "row_bytes must be a positive multiple of 4");
+    const uintptr_t al = (row_bytes % 16 == 0) ? 15u : 3u;
+    if (((uintptr_t)src | (uintptr_t)dst) & al)
+      return fail(MMSP_EINVAL, "src/dst must be %d-byte aligned for row_bytes %lld", (int)al + 1, (long long)row_bytes);
     const char* s = static_cast<const char*>(src);
     const char* e = static_cast<const char*>(dst);
     const int64_t bytes = N * row_bytes;
@@ -184,8 +186,13 @@ int mmsp_shard(const int32_t* seg_len, const uint8_t* seg_kind, int32_t n_seg, i
   if (src) {
     int64_t blocks = (N + 7) / 8;  // 8 warps (rows) per block
     if (blocks > 16LL * sms) blocks = 16LL * sms;
-    shard_rows_kernel<<<(unsigned)blocks, 256, 0, st>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst),
-                                                         (int32_t)N, P, row_bytes / 16, inverse ? 1 : 0);
+    if (row_bytes % 16 == 0)
+      shard_rows_kernel<<<(unsigned)blocks, 256, 0, st>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst),
+                                                           (int32_t)N, P, row_bytes / 16, inverse ? 1 : 0);
+    else
+      shard_rows_words_kernel<<<(unsigned)blocks, 256, 0, st>>>(static_cast<const uint32_t*>(src),
+                                                                 static_cast<uint32_t*>(dst), (int32_t)N, P,
+                                                                 row_bytes / 4, inverse ? 1 : 0);
     MMSP_CUDA(cudaGetLastError());
   }
   return ok();

@@ -122,4 +122,20 @@ __global__ void __launch_bounds__(256) shard_rows_kernel(const uint4* __restrict
   }
 }
 
+// Same permute for rows whose length is a multiple of 4 bytes only.
+__global__ void __launch_bounds__(256) shard_rows_words_kernel(const uint32_t* __restrict__ src,
+                                                               uint32_t* __restrict__ dst, int32_t N, int32_t P,
+                                                               int64_t row_words, int inverse) {
+  const int64_t C = N / (2 * P);
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t l = warp; l < N; l += nwarps) {
+    const int64_t g = zigzag_global(l, C, P);
+    const uint32_t* s = src + (inverse ? l : g) * row_words;
+    uint32_t* d = dst + (inverse ? g : l) * row_words;
+    for (int64_t i = lane; i < row_words; i += 32) d[i] = __ldg(s + i);
+  }
+}
+
 }  // namespace mmsp

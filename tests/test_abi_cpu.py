@@ -65,7 +65,8 @@ def test_shard_rejects_bad_arguments():
     _einval(m.mmsp_shard, np.ones(4097, np.int32), np.zeros(4097, np.uint8), 4097 * 2, 1,
             rank_counts=p)                                                     # over capacity
     _einval(m.mmsp_shard, None, None, 8, 2, src=p, dst=None)                  # half a permute
-    _einval(m.mmsp_shard, None, None, 8, 2, src=p, dst=p + 4096, row_bytes=24)  # row_bytes % 16
+    _einval(m.mmsp_shard, None, None, 8, 2, src=p, dst=p + 4096, row_bytes=6)  # row_bytes % 4
+    _einval(m.mmsp_shard, None, None, 8, 2, src=p + 4, dst=p + 4096, row_bytes=32)  # misaligned
     _einval(m.mmsp_shard, None, None, 8, 2, src=p, dst=p + 64, row_bytes=16)  # overlap
 
 

@@ -54,7 +54,7 @@ def test_segment_table_at_capacity():
     _assert_maps_equal(_maps(sl, sk, N, P), sharder.shard_maps(sl, sk, N, P))
 
 
-@pytest.mark.parametrize("N,P,row_bytes", [(4096, 4, 512), (1200, 3, 7168), (2, 1, 16), (65536, 32, 1024)])
+@pytest.mark.parametrize("N,P,row_bytes", [(4096, 4, 512), (1200, 3, 7168), (2, 1, 16), (65536, 32, 1024), (600, 1, 8), (1200, 3, 112), (144, 2, 28)])
 def test_row_permute_bit_exact_and_inverse(N, P, row_bytes):
     m = lib()
     g = torch.Generator(device="cuda").manual_seed(N)
