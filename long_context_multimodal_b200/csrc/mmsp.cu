@@ -327,13 +327,106 @@ extern "C" int mmsp_selftest_bounded_wait(int64_t max_cycles, void* stream) {
   return ok();
 }
 
+namespace {
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct BwdLayout {
+  int64_t C, Cp;
+  size_t vec_bytes, acc_bytes, total;
+};
+
+BwdLayout bwd_layout(int64_t N, int32_t P, int32_t Hq, int32_t d) {
+  BwdLayout L;
+  L.C = N / (2 * (int64_t)P);
+  L.Cp = (L.C + 127) / 128 * 128;
+  L.vec_bytes = align256((size_t)Hq * 2 * P * L.Cp * sizeof(float));
+  L.acc_bytes = align256((size_t)N * Hq * d * sizeof(float));
+  L.total = 2 * L.vec_bytes + L.acc_bytes;
+  return L;
+}
+}  // namespace
+
 extern "C" size_t mmsp_bwd_workspace_bytes(int64_t N, int32_t P, int32_t Hq, int32_t d) {
-  (void)N; (void)P; (void)Hq; (void)d;
-  return 0;
+  if (N <= 0 || P < 1 || Hq < 1 || d < 1 || N % (2 * (int64_t)P)) return 0;
+  return bwd_layout(N, P, Hq, d).total;
 }
 
-extern "C" int mmsp_attn_bwd(const void*, const void*, const void*, const void*, const void*, const float*, int64_t,
-                             int32_t, int32_t, int32_t, int32_t, float, int32_t, void*, void*, void*, float*, void*,
-                             size_t, void*) {
-  return fail(MMSP_EUNSUPPORTED, "backward not built yet");
+extern "C" int mmsp_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                             const float* lse, int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d, float scale,
+                             int32_t causal, void* dq, void* dk, void* dv, float* dq_acc_opt, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  int rc = check_common(N, P);
+  if (rc) return rc;
+  if ((rc = check_heads(Hq, Hkv, d))) return rc;
+  if (d != 128) return fail(MMSP_EUNSUPPORTED, "mmsp_attn_bwd supports d = 128 (got %d)", d);
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(MMSP_EINVAL, "scale must be finite and > 0");
+  if (causal != 0 && causal != 1) return fail(MMSP_EINVAL, "causal must be 0 or 1");
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv)
+    return fail(MMSP_EINVAL, "q, k, v, o, dout, lse, dq, dk, dv must be non-NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (dq_acc_opt && !aligned16(dq_acc_opt)))
+    return fail(MMSP_EINVAL, "all tensors must be 16-byte aligned");
+  if (N == 0) return ok();
+  const BwdLayout Lw = bwd_layout(N, P, Hq, d);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(MMSP_EINVAL, "workspace must be non-NULL and 256-byte aligned");
+  if (workspace_bytes < Lw.total)
+    return fail(MMSP_EINVAL, "workspace too small: %zu < %zu bytes", workspace_bytes, Lw.total);
+  int dev, sms;
+  if ((rc = current_device(&dev)) || (rc = device_sms(dev, &sms)) || (rc = get_encode())) return rc;
+  CUtensorMap tq, tk, tv, tdo;
+  if ((rc = tmap_rows_heads(&tq, q, N, Hq, d)) || (rc = tmap_rows_heads(&tk, k, N, Hkv, d)) ||
+      (rc = tmap_rows_heads(&tv, v, N, Hkv, d)) || (rc = tmap_rows_heads(&tdo, dout, N, Hq, d)))
+    return rc;
+  char* ws = static_cast<char*>(workspace);
+  float* lse2t = reinterpret_cast<float*>(ws);
+  float* dt = reinterpret_cast<float*>(ws + Lw.vec_bytes);
+  float* acc = dq_acc_opt ? dq_acc_opt : reinterpret_cast<float*>(ws + 2 * Lw.vec_bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  const int64_t pre_warps = (int64_t)P * 2 * Lw.Cp * Hq;
+  int64_t pre_blocks = (pre_warps + 7) / 8;
+  if (pre_blocks > 16LL * sms) pre_blocks = 16LL * sms;
+  bwd::bwd_pre_kernel<<<(unsigned)pre_blocks, 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2t, dt, acc, P, Hq,
+      Lw.C, Lw.Cp, 1);
+  MMSP_CUDA(cudaGetLastError());
+
+  bwd::Params p;
+  p.P = P;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.C = Lw.C;
+  p.Cp = Lw.Cp;
+  p.ntiles = (int32_t)(Lw.Cp / 128);
+  p.causal = causal;
+  p.n_units = 2LL * P * p.ntiles * Hkv;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale = scale;
+  p.lse2t = lse2t;
+  p.dt = dt;
+  p.dq_acc = acc;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.wait_cap = kWaitCapCycles;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_dev[dev].bwd_attr[1]) {
+      MMSP_CUDA(cudaFuncSetAttribute(bwd::attn_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     bwd::Smem::ALLOC));
+      g_dev[dev].bwd_attr[1] = true;
+    }
+  }
+  const int64_t grid = p.n_units < sms ? p.n_units : sms;
+  bwd::attn_bwd_kernel<<<(unsigned)grid, bwd::kThreads, bwd::Smem::ALLOC, st>>>(tq, tk, tv, tdo, p);
+  MMSP_CUDA(cudaGetLastError());
+
+  const int64_t n4 = N * Hq * d / 4;
+  int64_t cblocks = (n4 + 255) / 256;
+  if (cblocks > 16LL * sms) cblocks = 16LL * sms;
+  bwd::bwd_dq_convert_kernel<<<(unsigned)cblocks, 256, 0, st>>>(reinterpret_cast<const float4*>(acc),
+                                                                 static_cast<uint2*>(dq), n4);
+  MMSP_CUDA(cudaGetLastError());
+  return ok();
 }

@@ -202,31 +202,37 @@ def attention_bwd_rows(q_rows, k, v, do_rows, rows, scale=None, block: int = 64)
     return {"O": O, "LSE": LSE, "dQ": dQ}
 
 
-def attention_bwd_keys(q, k, v, do, keys, scale=None, block: int = 64):
+def attention_bwd_keys(q_tail, k, v, do_tail, keys, scale=None, block: int = 64):
     """dK and dV for selected global key positions.
 
-    Key j receives contributions from rows i >= j only, so this computes the
-    rows [min(keys), N) in full (their LSE and D) and sums their terms into
-    the requested keys. Cheap only when the keys lie near the end.
+    Key j receives contributions from rows i >= j only. q_tail and do_tail
+    hold the rows [j0, N) of Q and dO, where j0 = min(keys) and N = len(k);
+    those rows are computed in full (their LSE and D over keys <= i) and
+    their terms are summed into the requested keys. Cheap only when the keys
+    lie near the end.
     """
-    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     keys = np.asarray(keys, np.int64)
-    N, hq, d = q.shape
+    N = k.shape[0]
     hkv = k.shape[1]
+    hq, d = q_tail.shape[1], q_tail.shape[2]
+    j0 = int(keys.min())
+    if q_tail.shape[0] != N - j0 or do_tail.shape[0] != N - j0:
+        raise ValueError("q_tail/do_tail must hold rows [min(keys), N)")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    j0 = int(keys.min())
+    q_tail, do_tail = _f64(q_tail), _f64(do_tail)
     dK = np.zeros((len(keys), hkv, d))
     dV = np.zeros((len(keys), hkv, d))
-    for h in range(hq):
-        kh = kv_head(h, hq, hkv)
-        for i0 in range(j0, N, block):
-            rows = np.arange(i0, min(N, i0 + block))
-            _, _, _, _, p, ds = _rows_backward(q[rows, h], do[rows, h], rows,
-                                               k[:, kh], v[:, kh], scale)
-            pk = p[:, keys[keys <= rows.max()]]
-            dsk = ds[:, keys[keys <= rows.max()]]
-            sel = np.nonzero(keys <= rows.max())[0]
-            dV[sel, kh] += pk.T @ do[rows, h]
-            dK[sel, kh] += scale * (dsk.T @ q[rows, h])
+    for kh in range(hkv):
+        K = _f64(k[:, kh])
+        V = _f64(v[:, kh])
+        for h in range(hq):
+            if kv_head(h, hq, hkv) != kh:
+                continue
+            for i0 in range(j0, N, block):
+                rows = np.arange(i0, min(N, i0 + block))
+                _, _, _, _, p, ds = _rows_backward(q_tail[rows - j0, h], do_tail[rows - j0, h], rows, K, V, scale)
+                sel = np.nonzero(keys <= rows.max())[0]
+                dV[sel, kh] += p[:, keys[sel]].T @ do_tail[rows - j0, h]
+                dK[sel, kh] += scale * (ds[:, keys[sel]].T @ q_tail[rows - j0, h])
     return {"dK": dK, "dV": dV}

@@ -82,3 +82,39 @@ def check_bf16_rounding(o_out, o_acc):
     a = o_out.view(torch.int16).to(torch.int32)
     b = ref.view(torch.int16).to(torch.int32)
     assert int((a - b).abs().max()) <= 1
+
+
+# Gradient bars (a reading; none is stated for the backward): per tensor,
+# max|g - g_ref| / max(1, max|g_ref|) <= 1e-2 and mean|g - g_ref| / mean|g_ref|
+# <= 1e-2, on the fp32/bf16 outputs against the fp64 oracle.
+G_MAX_REL = 1e-2
+G_MEAN_REL = 1e-2
+
+
+def compare_grad(g, g_ref, what):
+    g = np.asarray(g, np.float64)
+    g_ref = np.asarray(g_ref, np.float64)
+    assert np.isfinite(g).all(), what + ": non-finite"
+    err = np.abs(g - g_ref)
+    mx = err.max() / max(1.0, np.abs(g_ref).max())
+    mn = err.mean() / max(np.abs(g_ref).mean(), 1e-30)
+    assert mx <= G_MAX_REL, f"{what}: max rel {mx:.3e}"
+    assert mn <= G_MEAN_REL, f"{what}: mean rel {mn:.3e}"
+    return float(mx), float(mn)
+
+
+def run_backward(ql, kl, vl, o_out, dol, lse, P, causal=1, fp32_dq=False):
+    """Rank-local inputs; returns (dq bf16, dk bf16, dv bf16, dq fp32 or None)."""
+    m = lib()
+    N, hq, d = ql.shape
+    hkv = kl.shape[1]
+    ws_bytes = m.mmsp_bwd_workspace_bytes(N, P, hq, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=ql.device)
+    dq = torch.full_like(ql, float("nan"))
+    dk = torch.full_like(kl, float("nan"))
+    dv = torch.full_like(vl, float("nan"))
+    dq32 = torch.full((N, hq, d), float("nan"), device=ql.device) if fp32_dq else None
+    m.mmsp_attn_bwd(ql, kl, vl, o_out, dol, lse, N, P, hq, hkv, d, 1.0 / math.sqrt(d), causal, dq, dk, dv, dq32,
+                    ws, ws_bytes)
+    m.mmsp_device_status()
+    return dq, dk, dv, dq32

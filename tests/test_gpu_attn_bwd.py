@@ -1,0 +1,118 @@
+"""Backward of the ring attention on the GPU (C ABI) against the fp64
+oracle: whole gradients at small sizes (ragged chunks, GQA ratios, one
+rank, non-causal), and at the full workload sizes sampled dQ rows, dK/dV of
+the last keys, and the closed-form gradient sums."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import mmsp_inputs as mi
+from oracle import attention as A
+from oracle import merge as M
+from gpu_util import (compare_attention, compare_grad, inputs, lib, needs_gpu, run_backward, run_forward,
+                      shard_rows)
+
+pytestmark = [pytest.mark.gpu, needs_gpu]
+
+
+def _fwd_bwd(q, k, v, do, P, causal=1, fp32_dq=False):
+    N = q.shape[0]
+    ql, kl, vl, dol = (shard_rows(x, N, P) for x in (q, k, v, do))
+    o_acc, lse, o_out = run_forward(ql, kl, vl, P, causal=causal)
+    dq, dk, dv, dq32 = run_backward(ql, kl, vl, o_out, dol, lse, P, causal=causal, fp32_dq=fp32_dq)
+    back = lambda x: shard_rows(x, N, P, inverse=True)
+    out = {"O": back(o_acc), "LSE": back(lse), "dQ": back(dq), "dK": back(dk), "dV": back(dv)}
+    if dq32 is not None:
+        out["dQ32"] = back(dq32)
+    return out
+
+
+CASES = [
+    # N, P, Hq, Hkv
+    (1024, 2, 2, 1),
+    (1200, 3, 4, 2),   # C = 200: ragged key and query tiles
+    (600, 1, 2, 2),    # one rank
+    (144, 2, 7, 1),    # C = 36: chunk shorter than a tile
+    (2048, 8, 28, 4),  # C = 128, GQA 7:1
+    (2560, 4, 3, 1),   # C = 320
+]
+
+
+@pytest.mark.parametrize("N,P,hq,hkv", CASES)
+def test_backward_matches_oracle_whole_gradients(N, P, hq, hkv):
+    d = 128
+    _, q, k, v, do = inputs(N, hq, hkv, d, seed=3 * N + P, with_dout=True)
+    out = _fwd_bwd(q, k, v, do, P, fp32_dq=True)
+    ref = A.causal_attention_bwd(*(x.float().cpu().numpy() for x in (q, k, v, do)))
+    compare_attention(out["O"].cpu().numpy(), out["LSE"].cpu().numpy(), ref["O"], ref["LSE"], "fwd")
+    for name in ("dQ", "dK", "dV"):
+        compare_grad(out[name].float().cpu().numpy(), ref[name], f"{name} N={N} P={P}")
+    compare_grad(out["dQ32"].cpu().numpy(), ref["dQ"], "dQ fp32")
+    # bf16 dQ is the RNE rounding of the fp32 accumulator
+    assert torch.equal(out["dQ"].view(torch.int16), out["dQ32"].to(torch.bfloat16).view(torch.int16))
+
+
+def test_backward_non_causal():
+    N, P, hq, hkv, d = 512, 2, 2, 1, 128
+    _, q, k, v, do = inputs(N, hq, hkv, d, seed=77, with_dout=True)
+    out = _fwd_bwd(q, k, v, do, P, causal=0)
+    tq, tk, tv = (x.double().cpu().requires_grad_(True) for x in (q, k, v))
+    G = hq // hkv
+    o = torch.nn.functional.scaled_dot_product_attention(
+        tq.transpose(0, 1), tk.repeat_interleave(G, 1).transpose(0, 1),
+        tv.repeat_interleave(G, 1).transpose(0, 1)).transpose(0, 1)
+    o.backward(do.double().cpu())
+    for name, ref in (("dQ", tq.grad), ("dK", tk.grad), ("dV", tv.grad)):
+        compare_grad(out[name].float().cpu().numpy(), ref.numpy(), name + " non-causal")
+
+
+def _closed_forms(dk, dv, do, hkv):
+    """sum_j dV_j = sum_i sum_{h in group} dO_i,h ; sum_j dK_j = 0."""
+    N, hq, d = do.shape
+    G = hq // hkv
+    sdv = dv.double().sum(0)
+    sdo = do.double().view(N, hkv, G, d).sum((0, 2))
+    err_v = (sdv - sdo).abs().max().item() / max(1.0, sdo.abs().max().item())
+    sdk = dk.double().sum(0)
+    err_k = sdk.abs().max().item() / max(1.0, dk.double().abs().sum(0).max().item())
+    assert err_v <= 1e-3, f"sum dV mismatch {err_v:.3e}"
+    assert err_k <= 1e-3, f"sum dK not ~0 {err_k:.3e}"
+
+
+def _full_size(name, n_rows, n_keys):
+    w = mi.WORKLOADS[name]
+    q, k, v, do = mi.workload_tensors(w, device="cuda", with_dout=True)
+    out = _fwd_bwd(q, k, v, do, w.P)
+    _closed_forms(out["dK"], out["dV"], do, w.hkv)
+    rows = mi.sample_rows(w.N, w.C, n_rows, 3000 + w.index)
+    ridx = torch.as_tensor(rows, device="cuda")
+    keys = np.arange(w.N - n_keys, w.N)
+    kidx = torch.as_tensor(keys, device="cuda")
+    got = {"dQ": out["dQ"][ridx].float().cpu().numpy(), "LSE": out["LSE"][ridx].cpu().numpy(),
+           "dK": out["dK"][kidx].float().cpu().numpy(), "dV": out["dV"][kidx].float().cpu().numpy()}
+    qr, dor = q[ridx].float().cpu().numpy(), do[ridx].float().cpu().numpy()
+    del out
+    kc, vc = k.float().cpu().numpy(), v.float().cpu().numpy()
+    ref = A.attention_bwd_rows(qr, kc, vc, dor, rows)
+    np.testing.assert_allclose(got["LSE"], ref["LSE"], atol=1e-3)
+    compare_grad(got["dQ"], ref["dQ"], f"{name} dQ rows")
+    # dK/dV of the last keys need only the rows after them
+    qt = q[w.N - n_keys:].float().cpu().numpy()
+    dot = do[w.N - n_keys:].float().cpu().numpy()
+    refk = A.attention_bwd_keys(qt, kc, vc, dot, keys)
+    compare_grad(got["dK"], refk["dK"], f"{name} dK last keys")
+    compare_grad(got["dV"], refk["dV"], f"{name} dV last keys")
+
+
+def test_n128k_sampled_gradients():
+    _full_size("n128k", 1024, 256)
+
+
+def test_n512k_sampled_gradients():
+    _full_size("n512k", 256, 128)
+
+
+def test_n1m_sampled_gradients():
+    _full_size("n1m", 192, 64)

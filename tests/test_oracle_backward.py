@@ -80,6 +80,6 @@ def test_rows_and_keys_variants_equal_full():
     np.testing.assert_allclose(r["dQ"], g["dQ"][rows], atol=1e-12)
     np.testing.assert_allclose(r["LSE"], g["LSE"][rows], atol=1e-12)
     keys = np.array([60, 61, 75, 89])
-    kk = A.attention_bwd_keys(q, k, v, do, keys, block=7)
+    kk = A.attention_bwd_keys(q[60:], k, v, do[60:], keys, block=7)
     np.testing.assert_allclose(kk["dK"], g["dK"][keys], atol=1e-12)
     np.testing.assert_allclose(kk["dV"], g["dV"][keys], atol=1e-12)
