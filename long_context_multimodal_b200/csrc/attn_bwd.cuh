@@ -172,7 +172,10 @@ struct Smem {
   static constexpr int OFF_BAR = OFF_VEC + 2 * 1024;
   static constexpr int NBAR = 16;
   static constexpr int BYTES = OFF_BAR + NBAR * 8 + 16;
-  static constexpr int ALLOC = BYTES + 1024;
+  // No alignment slack fits next to seven 32 KB tiles: the kernel requires a
+  // 1024-byte aligned dynamic shared memory base (it is, when the kernel has
+  // no static shared memory) and reports a layout error otherwise.
+  static constexpr int ALLOC = BYTES;
 };
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
@@ -192,9 +195,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   using L = Smem;
   constexpr int D = 128;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t base = smem_u32(smem_raw);
+  if (base & 1023u) {
+    if (threadIdx.x == 0) atomicExch(&g_timeout_flag, 2);
+    return;
+  }
+  uint8_t* gbase = smem_raw;
   const uint32_t sK = base + L::OFF_K, sV = base + L::OFF_V;
   const uint32_t sQ0 = base + L::OFF_Q;
   const uint32_t sDO = base + L::OFF_DO;

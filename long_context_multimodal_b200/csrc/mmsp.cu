@@ -297,6 +297,7 @@ int mmsp_device_status(void* stream) {
   if (flag) {
     const int zero = 0;
     MMSP_CUDA(cudaMemcpyToSymbol(g_timeout_flag, &zero, sizeof(int)));
+    if (flag == 2) return fail(MMSP_ECUDA, "a kernel found its shared memory base misaligned and did nothing");
     return fail(MMSP_ETIMEOUT, "a bounded device-side wait gave up");
   }
   return ok();

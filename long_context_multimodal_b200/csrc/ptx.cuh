@@ -10,8 +10,9 @@
 
 namespace mmsp {
 
-// Recorded by any kernel whose bounded wait gives up; read and cleared by
-// mmsp_device_status() on the host.
+// Device-side error word, read and cleared by mmsp_device_status() on the
+// host: 1 = a bounded wait gave up, 2 = a kernel found its shared memory
+// layout unusable and returned without work.
 __device__ int g_timeout_flag = 0;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

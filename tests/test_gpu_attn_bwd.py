@@ -69,16 +69,20 @@ def test_backward_non_causal():
 
 
 def _closed_forms(dk, dv, do, hkv):
-    """sum_j dV_j = sum_i sum_{h in group} dO_i,h ; sum_j dK_j = 0."""
+    """sum_j dV_j = sum_i sum_{h in group} dO_i,h and sum_j dK_j = 0 (each row
+    of dS sums to zero). dK, dV are bf16 (relative rounding <= 2^-9 each), so
+    the sums may differ from the exact values by at most 2^-9 sum_j |g_j|
+    plus the fp32 accumulation error inside the kernel; the bar is twice the
+    rounding bound."""
     N, hq, d = do.shape
     G = hq // hkv
     sdv = dv.double().sum(0)
     sdo = do.double().view(N, hkv, G, d).sum((0, 2))
-    err_v = (sdv - sdo).abs().max().item() / max(1.0, sdo.abs().max().item())
+    bound_v = 2.0 ** -8 * dv.double().abs().sum(0)
+    assert bool(((sdv - sdo).abs() <= bound_v + 1e-6).all()), "sum dV != sum dO"
     sdk = dk.double().sum(0)
-    err_k = sdk.abs().max().item() / max(1.0, dk.double().abs().sum(0).max().item())
-    assert err_v <= 1e-3, f"sum dV mismatch {err_v:.3e}"
-    assert err_k <= 1e-3, f"sum dK not ~0 {err_k:.3e}"
+    bound_k = 2.0 ** -8 * dk.double().abs().sum(0)
+    assert bool((sdk.abs() <= bound_k + 1e-6).all()), "sum dK != 0"
 
 
 def _full_size(name, n_rows, n_keys):
