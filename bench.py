@@ -1,0 +1,413 @@
+"""Benchmark: ring-blockwise causal attention (MM-SP hot path) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload n512k] [--impl reference]
+
+One step is one pass of the whole hot path over one synthetic sequence:
+zigzag shard maps, gather of Q/K/V/dO into rank-local order, attention
+forward over every virtual rank and ring step (merge fused), backward, and
+the inverse scatter of O/dQ/dK/dV -- all through the C ABI of libmmsp.so.
+Throughput is algorithmic causal flops (forward 4*d*Hq*N(N+1)/2, forward +
+backward 3.5x that) per second.
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent
+sequence (weak scaling, no collective on the data path); time is the max
+over ranks. `--impl reference` times the fp64 CPU oracle on a bounded row
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import signal
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import mmsp_inputs as mi  # noqa: E402
+
+METRIC = "causal ring-attention TFLOP/s fwd & fwd+bwd at N=32K–1M; % of B200 BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash(names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "long_context_multimodal_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(profile_md, source_files):
+    """Per-launch DRAM bytes recorded from an ncu capture, or None when the
+    summary is missing or the kernel source changed since the capture."""
+    path = os.path.join(ROOT, "profiles", profile_md)
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    s = re.search(r"source_sha:\s*([0-9a-f]+)", text)
+    if not m or not s or s.group(1) != kernel_source_hash(source_files):
+        return None
+    return float(m.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.send_signal(signal.SIGTERM)
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == 8:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
+        mx = [num(r[1]) for r in rows if num(r[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower().startswith("active")})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+_KV_CACHE = {}
+
+
+def cpu_sample_inputs(w, rows_count, seed):
+    """Rows of the workload for the CPU oracle without building all of Q:
+    K, V whole and Q, dO at the sampled rows (same recipe and distribution,
+    CPU generator)."""
+    import torch
+
+    rows = np.sort(np.random.default_rng(seed).choice(w.N, rows_count, replace=False))
+    g = torch.Generator().manual_seed(2000 + w.index + seed)
+    bf = lambda *s: torch.randn(s, generator=g).to(torch.bfloat16)
+    if w.name not in _KV_CACHE:
+        gk = torch.Generator().manual_seed(2000 + w.index)
+        vis = torch.as_tensor(mi.token_kinds(*mi.workload_layout(w)) == mi.VISUAL)
+        k = torch.randn((w.N, w.hkv, w.d), generator=gk).to(torch.bfloat16)
+        v = torch.randn((w.N, w.hkv, w.d), generator=gk).to(torch.bfloat16)
+        k[vis] = k[vis] * 2
+        _KV_CACHE[w.name] = (k.float().numpy(), v.float().numpy())
+    kc, vc = _KV_CACHE[w.name]
+    qr, dor = bf(rows_count, w.hq, w.d), bf(rows_count, w.hq, w.d)
+    return rows, qr.float().numpy(), kc, vc, dor.float().numpy()
+
+
+def oracle_sample(w, rows_count, seed, inputs=None):
+    """fp64 oracle (forward + dQ backward) on a bounded sample of query rows
+    of workload w; returns (algorithmic flops of the sample, seconds, threads)."""
+    import torch
+
+    from oracle import attention as A
+
+    rows, qr, kc, vc, dor = inputs if inputs is not None else cpu_sample_inputs(w, rows_count, seed)
+    t0 = time.perf_counter()
+    A.attention_bwd_rows(qr, kc, vc, dor, rows)
+    dt = time.perf_counter() - t0
+    # each sampled row i: forward 4*d*(i+1) flops per head, forward+backward 3.5x
+    flops = 3.5 * 4.0 * w.d * w.hq * float(np.sum(rows + 1))
+    return flops, dt, torch.get_num_threads()
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = mi.WORKLOADS[args.workload]
+    rows = args.ref_rows
+    sample = f"{rows} random query rows x all {w.hq} heads of {w.name} (N={w.N}): forward + dQ backward in fp64"
+    for i in range(args.warmup):
+        oracle_sample(w, max(4, rows // 8), 100 + i)
+    vals, secs = [], 0.0
+    threads = 1
+    for i in range(args.steps):
+        fl, dt, threads = oracle_sample(w, rows, 1000 + i)
+        vals.append(fl / dt / 1e12)
+        secs += dt
+    value = float(np.mean(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, gpus):
+    return {"workload": w.name, "N": w.N, "frames": w.frames, "frame_tokens": mi.FRAME_TOKENS,
+            "text_tokens": w.text_tokens, "text_segments": w.text_segments, "Hq": w.hq, "Hkv": w.hkv, "d": w.d,
+            "P_virtual_ranks": w.P, "causal": True, "global_batch": gpus, "seq_len": w.N,
+            "parallelism": f"{gpus} independent sequence(s), one per GPU; P virtual ranks per GPU",
+            "l2": "inputs larger than L2 (Q alone is N*Hq*d*2 bytes)"}
+
+
+def max_over_ranks(values, ws, device=None):
+    """Element-wise max of per-rank timings (the job takes as long as its
+    slowest rank)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def job_throughput(flops_per_step, ranks, ms_per_step):
+    """Whole-job TFLOP/s: every rank processes one sequence per step."""
+    return flops_per_step * ranks / (ms_per_step * 1e-3) / 1e12
+
+
+class Path:
+    """Device buffers and the C-ABI calls of one hot-path step."""
+
+    def __init__(self, w, device, seed_offset=0):
+        import torch
+
+        import long_context_multimodal_b200 as m
+
+        self.m = m
+        self.w = w
+        self.dev = device
+        N, P, hq, hkv, d = w.N, w.P, w.hq, w.hkv, w.d
+        self.seg_len, self.seg_kind = mi.workload_layout(w)
+        vis = mi.token_kinds(self.seg_len, self.seg_kind) == mi.VISUAL
+        self.q, self.k, self.v, self.do = mi.make_tensors(N, hq, hkv, d, 2000 + w.index + 100 * seed_offset, vis,
+                                                          device=device, with_dout=True)
+        e = lambda *s, dt=torch.bfloat16: torch.empty(s, dtype=dt, device=device)
+        self.ql, self.kl, self.vl, self.dol = e(N, hq, d), e(N, hkv, d), e(N, hkv, d), e(N, hq, d)
+        self.ol, self.dql, self.dkl, self.dvl = e(N, hq, d), e(N, hq, d), e(N, hkv, d), e(N, hkv, d)
+        self.o, self.dq, self.dk, self.dv = e(N, hq, d), e(N, hq, d), e(N, hkv, d), e(N, hkv, d)
+        self.lse = e(N, hq, dt=torch.float32)
+        self.l2g = e(N, dt=torch.int32)
+        self.g2l = e(N, dt=torch.int32)
+        self.mod = e(N, dt=torch.uint8)
+        self.segid = e(N, dt=torch.int32)
+        self.counts = e(P, 2, dt=torch.int32)
+        self.ws_bytes = m.mmsp_bwd_workspace_bytes(N, P, hq, d)
+        self.ws = e(self.ws_bytes, dt=torch.uint8)
+        self.scale = 1.0 / math.sqrt(d)
+        self.launches_per_step = 2 + 4 + 1 + 3 + 4
+
+    def step(self, stream, ev=None):
+        m, w = self.m, self.w
+        N, P = w.N, w.P
+        m.mmsp_shard(self.seg_len, self.seg_kind, N, P, self.l2g, self.g2l, self.mod, self.segid, self.counts,
+                     stream=stream)
+        for src, dst in ((self.q, self.ql), (self.k, self.kl), (self.v, self.vl), (self.do, self.dol)):
+            m.mmsp_shard(None, None, N, P, src=src, dst=dst, row_bytes=src[0].numel() * 2, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        m.mmsp_attn_fwd(self.ql, self.kl, self.vl, N, P, w.hq, w.hkv, w.d, self.scale, 1, 0, P, None, self.lse,
+                        self.ol, m.MMSP_FINALIZE, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        m.mmsp_attn_bwd(self.ql, self.kl, self.vl, self.ol, self.dol, self.lse, N, P, w.hq, w.hkv, w.d,
+                        self.scale, 1, self.dql, self.dkl, self.dvl, None, self.ws, self.ws_bytes, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        for src, dst in ((self.ol, self.o), (self.dql, self.dq), (self.dkl, self.dk), (self.dvl, self.dv)):
+            m.mmsp_shard(None, None, N, P, src=src, dst=dst, row_bytes=src[0].numel() * 2, inverse=True,
+                         stream=stream)
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+    w = mi.WORKLOADS[args.workload]
+    path = Path(w, dev, seed_offset=rank)
+    m = path.m
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        path.step(stream)
+    m.mmsp_device_status(stream)
+
+    # ---------------- device-resident timing
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
+    sampler = ClockSampler(cvd.split(",")[local] if cvd else local)
+    if rank == 0:
+        sampler.start()
+    barrier()
+    t_start.record(stream)
+    for i in range(args.steps):
+        path.step(stream, evs[i])
+    t_end.record(stream)
+    barrier()
+    clocks = sampler.stop() if rank == 0 else None
+    m.mmsp_device_status(stream)
+    ms_total = t_start.elapsed_time(t_end)
+    fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    ok = bool(torch.isfinite(path.dq.float()).all()) and bool(torch.isfinite(path.o.float()).all())
+
+    # ---------------- end to end through the C ABI with host buffers
+    pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+    h_in = [pin(t) for t in (path.q, path.k, path.v, path.do)]
+    for h, t in zip(h_in, (path.q, path.k, path.v, path.do)):
+        h.copy_(t)
+    h_out = [pin(t) for t in (path.o, path.dq, path.dk, path.dv)]
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+    e_steps = max(1, args.e2e_steps if args.e2e_steps is not None else args.steps)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        for h, t in zip(h_in, (path.q, path.k, path.v, path.do)):
+            t.copy_(h, non_blocking=True)
+        path.step(stream)
+        for h, t in zip(h_out, (path.o, path.dq, path.dk, path.dv)):
+            h.copy_(t, non_blocking=True)
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+    m.mmsp_device_status(stream)
+
+    # ---------------- max over ranks
+    ms_total, e2e_ms, fwd_ms, bwd_ms = max_over_ranks([ms_total, e2e_ms, fwd_ms, bwd_ms], ws, dev)
+    ms_step = ms_total / args.steps
+    flops = w.fwd_bwd_flops()
+    value = job_throughput(flops, ws, ms_step)
+    if rank == 0:
+        peaks, src = load_peaks()
+        peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        bwd_flops = 2.5 * w.fwd_flops()
+        achieved = bwd_flops / (bwd_ms * 1e-3) / 1e12
+        traffic = profiled_traffic(f"attn_bwd_{w.name}.md", ["attn_bwd.cuh", "ptx.cuh"])
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w, ws),
+            "fwd_tflops": w.fwd_flops() / (fwd_ms * 1e-3) / 1e12,
+            "fwd_bwd_tflops": value / ws,
+            "frac_of_bf16_peak": {"fwd": w.fwd_flops() / (fwd_ms * 1e-3) / 1e12 / peak,
+                                  "fwd_bwd": value / ws / peak, "peak_tflops": peak,
+                                  "peak_kind": f"bf16_tflops_sustained ({src})"},
+            "roofline": {"kernel": "attn_bwd (mmsp_attn_bwd: D preprocess + tcgen05 main + dQ convert)",
+                         "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"MEASURED_PEAKS.json bf16_tflops_sustained ({src})"},
+            "e2e": {"value": flops * ws / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": path.launches_per_step * args.steps,
+            "clocks": clocks,
+            "outputs_finite": ok,
+        }
+        if ws == 1 and not args.no_cpu_baseline:
+            rows = np.sort(np.random.default_rng(7).choice(w.N, args.ref_rows, replace=False))
+            ridx = torch.as_tensor(rows, device=dev)
+            inp = (rows, path.q[ridx].float().cpu().numpy(), path.k.float().cpu().numpy(),
+                   path.v.float().cpu().numpy(), path.do[ridx].float().cpu().numpy())
+            fl, dt, threads = oracle_sample(w, args.ref_rows, 7, inputs=inp)
+            line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                    "sample": f"{args.ref_rows} random query rows x {w.hq} heads of {w.name}: "
+                                              f"fp64 forward + dQ backward ({dt:.1f} s)"}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="n512k", choices=list(mi.WORKLOADS))
+    ap.add_argument("--impl", default="mmsp", choices=["mmsp", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=48)
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
