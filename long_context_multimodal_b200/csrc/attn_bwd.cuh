@@ -19,15 +19,15 @@
 //   dP^T = V dO^T                                     -> TMEM region SP
 //   dV  += P^T dO         (A = P^T from smem)         -> TMEM dV
 //   dK  += dS^T Q         (A = dS^T from smem)        -> TMEM dK
-//   dQ^T = K^T dS^T       (128 d x 128 queries)       -> TMEM dQ^T
-// dQ^T is read by four warps (one TMEM lane = one of d) and added into a
-// fp32 dQ accumulator with coalesced fp32 reductions; dK, dV are written
-// once per unit. Units are ordered by decreasing work (keys of chunk 0
+//   dQ   = dS K           (A = dS^T read MN-major)    -> TMEM dQ
+// dQ is read by four warps (one TMEM lane = one query row) and added into
+// a fp32 dQ accumulator with 16-byte vector reductions (red.add.v4.f32);
+// dK, dV are written once per unit. Units are ordered by decreasing work (keys of chunk 0
 // first).
 //
 // Warp roles (320 threads): warp 0 TMA producer, warp 1 MMA issuer, warps
 // 2-5 softmax/gradient (one thread per key = TMEM lane), warps 6-9 dQ
-// readout. TMEM: SP [0,128) dV [128,256) dK [256,384) dQ^T [384,512).
+// readout. TMEM: SP [0,128) dV [128,256) dK [256,384) dQ [384,512).
 // Shared memory: K, V (32 KB each), two Q stages, one dO stage, P^T and
 // dS^T (32 KB each), two 1 KB stages of LSE*log2(e) and D.
 #pragma once
@@ -184,8 +184,9 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
                : "memory");
 }
 
-__device__ __forceinline__ void red_add_f32(float* addr, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
+__device__ __forceinline__ void red_add_v4_f32(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -300,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idKQ = idesc_bf16_f32(BM, BN, 0, 0);   // S^T, dP^T
       constexpr uint32_t idGrad = idesc_bf16_f32(BM, D, 0, 1);  // dV, dK: B MN-major
-      constexpr uint32_t idDQ = idesc_bf16_f32(D, BN, 1, 1);    // dQ^T: A and B MN-major
+      constexpr uint32_t idDQ = idesc_bf16_f32(BN, D, 1, 1);    // dQ: A and B MN-major
       const uint32_t tSP = tmem, tDV = tmem + 128u, tDK = tmem + 256u, tDQ = tmem + 384u;
       uint32_t ucnt = 0, vis = 0, spf = 0, pc = 0, dqc = 0, epi = 0;
       auto issue_kq = [&](uint32_t a, uint32_t b) {  // tSP = a[128 x d] * b[128 x d]^T
@@ -372,14 +373,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         (kk > 0 || !first) ? 1u : 0u);
           }
           mma_commit(q_empty(st));
-          // dQ^T = K^T dS^T: A = K (MN-major: d contiguous), B = dS^T (MN-major: queries contiguous)
+          // dQ = dS K: A = dS^T tile read MN-major (queries contiguous, rows =
+          // keys), B = K tile read MN-major (d contiguous, rows = keys)
           if (dqc > 0) {
             mbar_wait(dq_free, (dqc - 1) & 1, abort_flag, cap);
             tc_fence_after();
           }
 #pragma unroll
           for (int kk = 0; kk < BM / 16; ++kk)
-            mma_bf16_ss(tDQ, desc_mnmajor_sw128(sK + kk * 2048, HALF), desc_mnmajor_sw128(sDST + kk * 2048, HALF),
+            mma_bf16_ss(tDQ, desc_mnmajor_sw128(sDST + kk * 2048, HALF), desc_mnmajor_sw128(sK + kk * 2048, HALF),
                         idDQ, kk > 0 ? 1u : 0u);
           mma_commit(dq_full);
           mma_commit(mm_done);
@@ -425,19 +427,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         uint32_t pk[64];  // P^T row as packed bf16 pairs
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t sr[64];
-          tmem_ld32(tSP + 64u * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-          tmem_ld32(tSP + 64u * h + 32u, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        for (int h = 0; h < 4; ++h) {
+          uint32_t sr[32];
+          tmem_ld32(tSP + 32u * h, sr);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 64; j += 2) {
-            const int c = 64 * h + j;
+          for (int j = 0; j < 32; j += 2) {
+            const int c = 32 * h + j;
             float e0 = ex2_approx(fmaf(__uint_as_float(sr[j]), sl2, -lse2[c]));
             float e1 = ex2_approx(fmaf(__uint_as_float(sr[j + 1]), sl2, -lse2[c + 1]));
             if (c < cmin) e0 = 0.f;
             if (c + 1 < cmin) e1 = 0.f;
-            pk[32 * h + j / 2] = pack_bf16x2(e0, e1);
+            pk[c / 2] = pack_bf16x2(e0, e1);
           }
         }
         tc_fence_before();
@@ -458,28 +459,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++spc;
         tc_fence_after();
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t sr[64];
-          tmem_ld32(tSP + 64u * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-          tmem_ld32(tSP + 64u * h + 32u, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        for (int h = 0; h < 4; ++h) {
+          uint32_t sr[32];
+          tmem_ld32(tSP + 32u * h, sr);
           tmem_wait_ld();
 #pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
+          for (int c8 = 0; c8 < 4; ++c8) {
+            const int c16 = 4 * h + c8;
+            const uint32_t off = (c16 >> 3) * HALF + row * 128 + ((((uint32_t)c16 & 7u) ^ ((uint32_t)row & 7u)) << 4);
+            uint32_t pv[4];  // this thread's own P^T values, read back from shared memory
+            ld_shared_v4(sPT + off, pv);
             uint32_t o[4];
 #pragma unroll
             for (int u2 = 0; u2 < 4; ++u2) {
               const int j = 8 * c8 + 2 * u2;
-              const int c = 64 * h + j;
-              const __nv_bfloat162 pp = *reinterpret_cast<const __nv_bfloat162*>(&pk[c / 2]);
+              const int c = 32 * h + j;
+              const __nv_bfloat162 pp = *reinterpret_cast<const __nv_bfloat162*>(&pv[u2]);
               const float p0 = __low2float(pp), p1 = __high2float(pp);
               const float d0 = p0 * (__uint_as_float(sr[j]) - dvec[c]);
               const float d1 = p1 * (__uint_as_float(sr[j + 1]) - dvec[c + 1]);
               o[u2] = pack_bf16x2(d0, d1);
             }
-            const int c16 = 8 * h + c8;
-            const uint32_t addr =
-                sDST + (c16 >> 3) * HALF + row * 128 + ((((uint32_t)c16 & 7u) ^ ((uint32_t)row & 7u)) << 4);
-            st_shared_v4(addr, o[0], o[1], o[2], o[3]);
+            st_shared_v4(sDST + off, o[0], o[1], o[2], o[3]);
           }
         }
         fence_proxy_async_smem();
@@ -524,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------ dQ readout
     const int wq = warp & 3;
-    const int dd = wq * 32 + lane;  // head-dim index = TMEM lane of dQ^T
+    const int row = wq * 32 + lane;  // query row of the tile = TMEM lane of dQ
     const uint32_t tDQ = tmem + 384u + ((uint32_t)(wq * 32) << 16);
     const float sc = p.scale;
     uint32_t dqc = 0;
@@ -535,23 +536,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(dq_full, dqc & 1, abort_flag, cap);
         ++dqc;
         tc_fence_after();
-        const int64_t nvalid = p.C - it.q0;  // queries of the tile inside the chunk
-        float* base_ptr = p.dq_acc + (it.lrow0 * p.Hq + it.h) * D + dd;
-        const int64_t rstride = (int64_t)p.Hq * D;
+        const bool row_ok = it.q0 + row < p.C;  // query inside the chunk
+        float* dst = p.dq_acc + ((it.lrow0 + row) * p.Hq + it.h) * D;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           uint32_t a[32];
           tmem_ld32(tDQ + 32u * c, a);
           tmem_wait_ld();
-          if (c == BN / 32 - 1) {
+          if (c == D / 32 - 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(dq_free);
           }
+          if (row_ok) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int q = 32 * c + j;
-            if (q < nvalid) red_add_f32(base_ptr + q * rstride, __uint_as_float(a[j]) * sc);
+            for (int j = 0; j < 32; j += 4)
+              red_add_v4_f32(dst + 32 * c + j, __uint_as_float(a[j]) * sc, __uint_as_float(a[j + 1]) * sc,
+                             __uint_as_float(a[j + 2]) * sc, __uint_as_float(a[j + 3]) * sc);
           }
         }
       }
