@@ -1,6 +1,8 @@
 """Build libmmsp.so (the sm_100a CUDA library behind include/mmsp.h) in-tree.
 
-    python -m long_context_multimodal_b200.build
+    python long_context_multimodal_b200/build.py [--force] [-v]
+
+(Run it as a file, not with -m: importing the package loads the library.)
 
 nvcc cross-compiles for sm_100a without a GPU. The shared library is written
 next to this file, where the Python binding loads it from.
