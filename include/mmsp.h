@@ -174,6 +174,46 @@ int mmsp_attn_bwd(const void* q, const void* k, const void* v,
 /* Scratch bytes mmsp_attn_bwd needs for these sizes (0 on invalid sizes). */
 size_t mmsp_bwd_workspace_bytes(int64_t N, int32_t P, int32_t Hq, int32_t d);
 
+/* Capacity of the library-owned scratch used by mmsp_attn_bwd_noalloc. */
+#define MMSP_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/*
+ * mmsp_attn_bwd_noalloc -- mmsp_attn_bwd for callers that cannot allocate
+ * device memory. (No counterpart on the pages: this is an interface
+ * convenience of this library.)
+ *
+ * Some callers own no allocator of their own or must not use one: code
+ * embedded in a host framework whose device memory is all handed out by
+ * that framework's pool (a cudaMalloc behind its back breaks its
+ * accounting), and latency-bound paths where cudaMalloc/cudaFree, which can
+ * synchronise the device, are not acceptable between launches. This entry
+ * point takes the same inputs and outputs as mmsp_attn_bwd but no
+ * workspace: its scratch (the padded LSE/D rows and the fp32 dQ
+ * accumulator) lives in one file-scope device array of
+ * MMSP_NOALLOC_SCRATCH_BYTES (64 MiB) inside libmmsp.so, which every GPU
+ * that loads the library keeps until the process exits.
+ *
+ *   Arguments as mmsp_attn_bwd, without workspace / workspace_bytes.
+ *   Sizes whose mmsp_bwd_workspace_bytes() exceeds the capacity are
+ *   rejected with MMSP_EINVAL (nothing launched); for example Hq = 28,
+ *   d = 128, N = 4096 needs about 60 MB and fits, N = 4608 does not.
+ *   The first call on a device resolves the array's device address on that
+ *   device (cudaGetSymbolAddress, with that device current); make that first
+ *   call before any stream capture. Later calls on the device reuse it.
+ *   The call allocates nothing (no cudaMalloc, cudaFree or allocating
+ *   library routine). All calls on a device share the one array and it keeps
+ *   the previous call's contents; everything the kernels need zeroed is
+ *   cleared inside the call. Calls that overlap on the GPU (different
+ *   streams, or different host threads on one device) race on the array and
+ *   must be serialised by the caller.
+ */
+int mmsp_attn_bwd_noalloc(const void* q, const void* k, const void* v,
+                          const void* o, const void* dout, const float* lse,
+                          int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d,
+                          float scale, int32_t causal,
+                          void* dq, void* dk, void* dv, float* dq_acc_opt,
+                          void* stream);
+
 /* Message of the calling thread's last failed call ("" if none). */
 const char* mmsp_last_error(void);
 

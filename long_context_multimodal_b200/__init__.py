@@ -14,6 +14,8 @@ from ._binding import (  # noqa: F401
     STATUS,
     lib_path,
     mmsp_attn_bwd,
+    mmsp_attn_bwd_noalloc,
+    MMSP_NOALLOC_SCRATCH_BYTES,
     mmsp_attn_fwd,
     mmsp_bwd_workspace_bytes,
     mmsp_device_status,

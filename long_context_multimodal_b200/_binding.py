@@ -31,7 +31,7 @@ def _load():
     if not os.path.exists(path):
         raise ImportError(
             f"{path} is missing: build the CUDA library first "
-            "(python -m long_context_multimodal_b200.build). There is no CPU fallback.")
+            "(python long_context_multimodal_b200/build.py). There is no CPU fallback.")
     return ctypes.CDLL(path)
 
 
@@ -48,6 +48,9 @@ _SIGS = {
                        c_int32, c_int32, c_float, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                        c_size_t, c_void_p], c_int32),
     "mmsp_bwd_workspace_bytes": ([c_int64, c_int32, c_int32, c_int32], c_size_t),
+    "mmsp_attn_bwd_noalloc": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32,
+                               c_int32, c_int32, c_int32, c_float, c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
+                               c_void_p], c_int32),
     "mmsp_last_error": ([], ctypes.c_char_p),
     "mmsp_device_status": ([c_void_p], c_int32),
     "mmsp_selftest_bounded_wait": ([c_int64, c_void_p], c_int32),
@@ -139,6 +142,19 @@ def mmsp_attn_bwd(q, k, v, o, dout, lse, N, P, Hq, Hkv, d, scale, causal, dq, dk
                             int(Hkv), int(d), float(scale), int(causal), _ptr(dq), _ptr(dk), _ptr(dv),
                             _ptr(dq_acc_opt), _ptr(workspace), int(workspace_bytes), _stream(stream))
     return _check("mmsp_attn_bwd", rc)
+
+
+def mmsp_attn_bwd_noalloc(q, k, v, o, dout, lse, N, P, Hq, Hkv, d, scale, causal, dq, dk, dv, dq_acc_opt,
+                          stream=None):
+    """Backward with the library's own fixed scratch (no allocation anywhere;
+    see include/mmsp.h for the capacity and the sharing rules)."""
+    rc = _lib.mmsp_attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), int(N), int(P),
+                                    int(Hq), int(Hkv), int(d), float(scale), int(causal), _ptr(dq), _ptr(dk),
+                                    _ptr(dv), _ptr(dq_acc_opt), _stream(stream))
+    return _check("mmsp_attn_bwd_noalloc", rc)
+
+
+MMSP_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 def mmsp_bwd_workspace_bytes(N, P, Hq, d) -> int:

@@ -431,3 +431,50 @@ extern "C" int mmsp_attn_bwd(const void* q, const void* k, const void* v, const 
   MMSP_CUDA(cudaGetLastError());
   return ok();
 }
+
+// ---------------------------------------------------------------------------
+// Allocation-free backward: the scratch of mmsp_attn_bwd in a file-scope
+// device array, shared by every call on a device.
+namespace {
+__device__ __align__(256) unsigned char g_bwd_scratch[MMSP_NOALLOC_SCRATCH_BYTES];
+
+void* g_scratch_ptr[kMaxDevices] = {};
+std::mutex g_scratch_mu;
+
+// Device address of g_bwd_scratch on the current device (host code only
+// sees a host-side stand-in for the symbol; passing that to a kernel would
+// be wrong). Resolved once per device.
+int scratch_address(int dev, void** out) {
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_bwd_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(MMSP_ECUDA, "cudaGetSymbolAddress(scratch) failed: %s", cudaGetErrorString(e));
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return MMSP_OK;
+}
+}  // namespace
+
+extern "C" int mmsp_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                     const float* lse, int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d,
+                                     float scale, int32_t causal, void* dq, void* dk, void* dv, float* dq_acc_opt,
+                                     void* stream) {
+  int rc = check_common(N, P);
+  if (rc) return rc;
+  if ((rc = check_heads(Hq, Hkv, d))) return rc;
+  if (N == 0) return mmsp_attn_bwd(q, k, v, o, dout, lse, N, P, Hq, Hkv, d, scale, causal, dq, dk, dv, dq_acc_opt,
+                                   nullptr, 0, stream);
+  const size_t need = mmsp_bwd_workspace_bytes(N, P, Hq, d);
+  if (need > (size_t)MMSP_NOALLOC_SCRATCH_BYTES)
+    return fail(MMSP_EINVAL, "sizes need %zu bytes of scratch; mmsp_attn_bwd_noalloc holds at most %zu (use "
+                "mmsp_attn_bwd with a caller workspace)", need, (size_t)MMSP_NOALLOC_SCRATCH_BYTES);
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  void* scratch = nullptr;
+  if ((rc = scratch_address(dev, &scratch))) return rc;
+  return mmsp_attn_bwd(q, k, v, o, dout, lse, N, P, Hq, Hkv, d, scale, causal, dq, dk, dv, dq_acc_opt, scratch,
+                       (size_t)MMSP_NOALLOC_SCRATCH_BYTES, stream);
+}

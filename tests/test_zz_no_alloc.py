@@ -1,0 +1,63 @@
+"""The allocation-free backward entry point (mmsp_attn_bwd_noalloc) against
+the workspace one (mmsp_attn_bwd), through the C ABI.
+
+Some callers of this library cannot allocate device memory: code running
+inside a host framework that hands out all device memory from its own pool,
+and latency-bound paths where a cudaMalloc/cudaFree (which can synchronise
+the device) is not acceptable. For them the backward keeps its scratch in a
+fixed array inside the library. This file is collected last on purpose: if
+it fails, a run that stops at the first failure has already run the rest.
+"""
+import math
+
+import pytest
+import torch
+
+from gpu_util import compare_grad, inputs, lib, needs_gpu, run_forward, shard_rows
+
+pytestmark = [pytest.mark.gpu, needs_gpu]
+
+
+def _case(N, P, hq, hkv, seed):
+    d = 128
+    _, q, k, v, do = inputs(N, hq, hkv, d, seed=seed, with_dout=True)
+    ql, kl, vl, dol = (shard_rows(x, N, P) for x in (q, k, v, do))
+    _, lse, o = run_forward(ql, kl, vl, P)
+    return ql, kl, vl, dol, o, lse
+
+
+def _grads(fn, ql, kl, vl, dol, o, lse, P, *extra):
+    m = lib()
+    N, hq, d = ql.shape
+    hkv = kl.shape[1]
+    dq, dk, dv = (torch.full_like(x, float("nan")) for x in (ql, kl, vl))
+    dq32 = torch.full(ql.shape, float("nan"), device=ql.device)
+    fn(ql, kl, vl, o, dol, lse, N, P, hq, hkv, d, 1.0 / math.sqrt(d), 1, dq, dk, dv, dq32, *extra)
+    m.mmsp_device_status()
+    return {"dQ": dq, "dK": dk, "dV": dv, "dQ32": dq32}
+
+
+def test_noalloc_backward_matches_workspace_backward_twice_in_a_row():
+    m = lib()
+    # two calls in a row with different sizes: the second must not see the
+    # first call's leftovers in the shared scratch
+    for N, P, hq, hkv, seed in ((4096, 4, 28, 4, 91), (1200, 3, 4, 2, 92)):
+        assert m.mmsp_bwd_workspace_bytes(N, P, hq, 128) <= m.MMSP_NOALLOC_SCRATCH_BYTES
+        args = _case(N, P, hq, hkv, seed)
+        got = _grads(m.mmsp_attn_bwd_noalloc, *args, P)
+        ws_bytes = m.mmsp_bwd_workspace_bytes(N, P, hq, 128)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+        ref = _grads(m.mmsp_attn_bwd, *args, P, ws, ws_bytes)
+        for name in ("dQ", "dK", "dV", "dQ32"):
+            compare_grad(got[name].float().cpu().numpy(), ref[name].float().cpu().numpy(),
+                         f"noalloc {name} N={N}")
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch():
+    m = lib()
+    N, P, hq = 8192, 4, 28
+    assert m.mmsp_bwd_workspace_bytes(N, P, hq, 128) > m.MMSP_NOALLOC_SCRATCH_BYTES
+    x = torch.zeros(16, device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(m.MmspError) as e:
+        m.mmsp_attn_bwd_noalloc(x, x, x, x, x, x, N, P, hq, 4, 128, 0.088, 1, x, x, x, None)
+    assert e.value.status == 1 and "scratch" in str(e.value)
