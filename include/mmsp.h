@@ -161,7 +161,9 @@ int mmsp_lse_merge(const float* o_a, const float* lse_a,
  *   dk, dv             DEVICE bf16 [P][2C][Hkv][d] (output)
  *   dq_acc_opt         DEVICE fp32 [P][2C][Hq][d] or NULL: fp32 dQ output.
  *   workspace          DEVICE scratch of at least mmsp_bwd_workspace_bytes()
- *                      bytes, 256-byte aligned; contents need not be zeroed.
+ *                      bytes (per-head LSE*log2(e) and D rows, about 8*Hq
+ *                      bytes per token), 256-byte aligned; contents need not
+ *                      be zeroed.
  *   d == 128 or 64; other constraints as mmsp_attn_fwd.
  */
 int mmsp_attn_bwd(const void* q, const void* k, const void* v,
@@ -188,15 +190,15 @@ size_t mmsp_bwd_workspace_bytes(int64_t N, int32_t P, int32_t Hq, int32_t d);
  * accounting), and latency-bound paths where cudaMalloc/cudaFree, which can
  * synchronise the device, are not acceptable between launches. This entry
  * point takes the same inputs and outputs as mmsp_attn_bwd but no
- * workspace: its scratch (the padded LSE/D rows and the fp32 dQ
- * accumulator) lives in one file-scope device array of
+ * workspace: its scratch (the padded per-head LSE/D rows) lives in one
+ * file-scope device array of
  * MMSP_NOALLOC_SCRATCH_BYTES (64 MiB) inside libmmsp.so, which every GPU
  * that loads the library keeps until the process exits.
  *
  *   Arguments as mmsp_attn_bwd, without workspace / workspace_bytes.
  *   Sizes whose mmsp_bwd_workspace_bytes() exceeds the capacity are
- *   rejected with MMSP_EINVAL (nothing launched); for example Hq = 28,
- *   d = 128, N = 4096 needs about 60 MB and fits, N = 4608 does not.
+ *   rejected with MMSP_EINVAL (nothing launched); for example with Hq = 28
+ *   N = 262,144 needs about 59 MB and fits, N = 524,288 does not.
  *   The first call on a device resolves the array's device address on that
  *   device (cudaGetSymbolAddress, with that device current); make that first
  *   call before any stream capture. Later calls on the device reuse it.

@@ -20,15 +20,18 @@
 //
 // Warp roles (320 threads, one CTA per SM):
 //   warp 0      TMA producer: Q tiles A/B once per item, then K_j, V_j into
-//               a 3-stage ring of 128 x d bf16 tiles (128-byte swizzle).
-//   warp 1      MMA issuer (one thread): S_X = Q_X K_j^T into TMEM, and
-//               O_X += P_X V_j with P_X from shared memory; ping-pong order
-//               PV_A(j), S_A(j+1), PV_B(j), S_B(j+1) so the tensor core works
-//               on one tile while the softmax warps work on the other.
+//               a 5-stage ring of 128 x d bf16 tiles (128-byte swizzle).
+//   warp 1      MMA issuer (warp-uniform, one lane issues): S_X = Q_X K_j^T
+//               into TMEM, and O_X += P_X V_j with P_X read from TMEM (the
+//               softmax writes bf16 P over the S columns it has consumed);
+//               ping-pong order PV_A(j), S_A(j+1), PV_B(j), S_B(j+1) so the
+//               tensor core works on one tile while the softmax warps work
+//               on the other. tcgen05 MMAs of one thread run in issue order,
+//               so S_X(j+1) overwrites P_X(j) only after PV_X(j) read it.
 //   warps 2-5   softmax for tile A, warps 6-9 for tile B: one thread per row
 //               (TMEM lane), fp32 online softmax in base 2, P written to
-//               shared memory as bf16, lazy O rescale (only when the running
-//               max grows by more than 2^8), epilogue O / l and LSE.
+//               TMEM as bf16, lazy O rescale (only when the running max grows
+//               by more than 2^8), epilogue O / l and LSE.
 // TMEM: S_A [0,128) S_B [128,256) O_A [256,256+d) O_B [256+d,256+2d).
 #pragma once
 
@@ -44,7 +47,7 @@ namespace fwd {
 
 constexpr int BM = 128;      // query rows per tile
 constexpr int BN = 128;      // keys per tile
-constexpr int NSTAGE = 3;    // K/V ring stages
+constexpr int NSTAGE = 5;    // K/V ring stages
 constexpr int kThreads = 320;
 constexpr int HALF = 128 * 128;  // bytes of one 128-row x 64-column bf16 half tile
 
@@ -165,10 +168,8 @@ template <int D>
 struct Smem {
   static constexpr int QT = BM * D * 2;   // one Q tile
   static constexpr int KT = BN * D * 2;   // one K or V tile (a ring stage)
-  static constexpr int PT = BM * BN * 2;  // one P tile
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_P = 2 * QT;
-  static constexpr int OFF_KV = OFF_P + 2 * PT;
+  static constexpr int OFF_KV = 2 * QT;
   static constexpr int OFF_BAR = OFF_KV + NSTAGE * KT;
   static constexpr int NBAR = 2 * NSTAGE + 2 + 5 * 2;
   static constexpr int BYTES = OFF_BAR + NBAR * 8 + 16;
@@ -187,7 +188,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* gbase = smem_raw + (base - raw);
 
   const uint32_t sQ0 = base + L::OFF_Q, sQ1 = sQ0 + L::QT;
-  const uint32_t sP0 = base + L::OFF_P, sP1 = sP0 + L::PT;
   const uint32_t sKV = base + L::OFF_KV;
   const uint32_t bar0 = base + L::OFF_BAR;
   auto kv_full = [&](int i) { return bar0 + 8u * i; };
@@ -234,21 +234,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
+    // The whole warp runs the (uniform) control flow; lane 0 issues.
+    {
+      const uint32_t leader = lane == 0 ? 1u : 0u;
+      if (lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+      }
       int64_t pos = 0;
       uint32_t qcnt = 0;
       for (int64_t idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
         const Item it = decode_item(p, idx);
         if (qcnt > 0) mbar_wait(q_empty, (qcnt - 1) & 1, abort_flag, cap);
-        mbar_arrive_expect_tx(q_full, (uint32_t)((it.validA ? 1 : 0) + (it.validB ? 1 : 0)) * L::QT);
+        mbar_arrive_expect_tx_w(leader, q_full, (uint32_t)((it.validA ? 1 : 0) + (it.validB ? 1 : 0)) * L::QT);
         const int rowA = (int)((int64_t)it.r * 2 * p.C + (int64_t)it.c * p.C + it.rowA0);
 #pragma unroll
         for (int hf = 0; hf < NH; ++hf) {
-          tma_load_3d(sQ0 + hf * HALF, &tmQ, q_full, hf * 64, it.h, rowA);
-          if (it.validB) tma_load_3d(sQ1 + hf * HALF, &tmQ, q_full, hf * 64, it.h, rowA + 128);
+          tma_load_3d_w(leader, sQ0 + hf * HALF, &tmQ, q_full, hf * 64, it.h, rowA);
+          if (it.validB) tma_load_3d_w(leader, sQ1 + hf * HALF, &tmQ, q_full, hf * 64, it.h, rowA + 128);
         }
         ++qcnt;
         TileIter ti(p, it);
@@ -258,11 +262,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int st = (int)(pos % NSTAGE);
             const uint32_t use = (uint32_t)(pos / NSTAGE);
             mbar_wait(kv_empty(st), (use & 1) ^ 1, abort_flag, cap);
-            mbar_arrive_expect_tx(kv_full(st), L::KT);
+            mbar_arrive_expect_tx_w(leader, kv_full(st), L::KT);
 #pragma unroll
             for (int hf = 0; hf < NH; ++hf)
-              tma_load_3d(sKV + st * L::KT + hf * HALF, kv ? (const void*)&tmV : (const void*)&tmK, kv_full(st),
-                          hf * 64, it.kvh, (int)ti.kv_row);
+              tma_load_3d_w(leader, sKV + st * L::KT + hf * HALF, kv ? (const void*)&tmV : (const void*)&tmK,
+                            kv_full(st), hf * 64, it.kvh, (int)ti.kv_row);
             ++pos;
           }
         }
@@ -275,13 +279,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the (uniform) control flow and computes the
+    // descriptors; lane 0 issues the tcgen05 instructions.
+    {
+      const uint32_t leader = lane == 0 ? 1u : 0u;
       constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(BM, D, 0, 1);
       const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
       const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
       const uint32_t sQ[2] = {sQ0, sQ1};
-      const uint32_t sP[2] = {sP0, sP1};
       const std::integral_constant<int, 0> kA{};
       const std::integral_constant<int, 1> kB{};
       int64_t pos = 0;
@@ -303,9 +309,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
-          mma_bf16_ss(tS[x], desc_kmajor_sw128(sQ[x] + off), desc_kmajor_sw128(sk + off), idS, kk > 0 ? 1u : 0u);
+          mma_bf16_ss_w(leader, tS[x], desc_kmajor_sw128(sQ[x] + off), desc_kmajor_sw128(sk + off), idS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(s_full(x));
+        mma_commit_w(leader, s_full(x));
         ++s_cnt[x];
       };
       auto issue_PV = [&](auto X, int64_t vpos) {
@@ -317,13 +323,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
         }
         const uint32_t sv = sKV + (uint32_t)(vpos % NSTAGE) * L::KT;
+        // P_X is in TMEM over the first 64 columns of S_X (8 columns = 16
+        // keys per instruction)
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint32_t aoff = (kk >> 2) * HALF + (kk & 3) * 32;
-          mma_bf16_ss(tO[x], desc_kmajor_sw128(sP[x] + aoff), desc_mnmajor_sw128(sv + kk * 2048, HALF), idO,
-                      (kk > 0 || !first_pv[x]) ? 1u : 0u);
-        }
-        mma_commit(o_done(x));
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_bf16_ts_w(leader, tO[x], tS[x] + 8u * kk, desc_mnmajor_sw128(sv + kk * 2048, HALF), idO,
+                        (kk > 0 || !first_pv[x]) ? 1u : 0u);
+        mma_commit_w(leader, o_done(x));
         ++pv_cnt[x];
         first_pv[x] = false;
       };
@@ -341,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           wait_full(kpos);
           if (ti.actA) issue_S(kA, kpos);
           if (ti.actB) issue_S(kB, kpos);
-          mma_commit(kv_empty((int)(kpos % NSTAGE)));
+          mma_commit_w(leader, kv_empty((int)(kpos % NSTAGE)));
         }
         while (has) {
           const bool curA = ti.actA, curB = ti.actB;
@@ -356,14 +362,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ti.actA) issue_S(kA, kn);
           }
           if (curB) issue_PV(kB, vpos);
-          mma_commit(kv_empty((int)(vpos % NSTAGE)));
+          mma_commit_w(leader, kv_empty((int)(vpos % NSTAGE)));
           if (has_next) {
             if (ti.actB) issue_S(kB, kn);
-            mma_commit(kv_empty((int)(kn % NSTAGE)));
+            mma_commit_w(leader, kv_empty((int)(kn % NSTAGE)));
           }
           has = has_next;
         }
-        mma_commit(q_empty);
+        mma_commit_w(leader, q_empty);
         if (!first_pv[0]) ++epi_cnt[0];
         if (!first_pv[1]) ++epi_cnt[1];
       }
@@ -376,7 +382,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + (uint32_t)(grp * 128) + lane_off;
     const uint32_t tO = tmem + 256u + (uint32_t)(grp * D) + lane_off;
-    const uint32_t sPx = grp ? sP1 : sP0;
     const float sl2 = p.scale_log2;
     uint32_t s_cnt = 0, pv_cnt = 0;
 
@@ -403,61 +408,82 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         // pass 1: row max over the tile, 64 columns per TMEM round trip
-        float mx = -CUDART_INF_F;
+        // The per-tile softmax, compiled twice: with the causal / ragged-tail
+        // mask (diagonal and last tiles) and without it (all other tiles).
+        float alpha = 1.f, rs = 0.f;
+        bool need = false;
+        auto tile = [&](auto MKc) {
+          constexpr bool MK = decltype(MKc)::value;
+          // eight independent max chains instead of one 128-long chain
+          float mxv[8];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t sr[64];
-          tmem_ld32(tS + 64u * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-          tmem_ld32(tS + 64u * h + 32u, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-          tmem_wait_ld();
+          for (int u = 0; u < 8; ++u) mxv[u] = -CUDART_INF_F;
 #pragma unroll
-          for (int j = 0; j < 64; ++j)
-            if (64 * h + j < lim) mx = fmaxf(mx, __uint_as_float(sr[j]));
-        }
-        const float mc = fmaxf(m, mx * sl2);
-        const bool need = mc > m + 8.0f;
-        float alpha = 1.f;
-        if (need) {
-          alpha = ex2_approx(m - mc);
-          m = mc;
-        }
-        const float mu = (m == -CUDART_INF_F) ? 0.f : m;
-        // The previous PV of this group is complete (it was issued before
-        // this S and tcgen05 work completes in order); the wait is cheap and
-        // makes the P buffer reuse explicit.
-        if (pv_cnt > 0) {
-          mbar_wait(o_done(grp), (pv_cnt - 1) & 1, abort_flag, cap);
-          tc_fence_after();
-        }
-        // pass 2: P = 2^(s*scale*log2e - m) as bf16 into the K-major,
-        // 128-byte-swizzled P tile (half h holds keys [64h, 64h+64)).
-        float rs = 0.f;
+          for (int h = 0; h < 2; ++h) {
+            uint32_t sr[64];
+            tmem_ld32(tS + 64u * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            tmem_ld32(tS + 64u * h + 32u, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+            tmem_wait_ld();
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t sr[64];
-          tmem_ld32(tS + 64u * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-          tmem_ld32(tS + 64u * h + 32u, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int j0 = 8 * c + 2 * u;
-              float e0 = ex2_approx(fmaf(__uint_as_float(sr[j0]), sl2, -mu));
-              float e1 = ex2_approx(fmaf(__uint_as_float(sr[j0 + 1]), sl2, -mu));
-              if (64 * h + j0 >= lim) e0 = 0.f;
-              if (64 * h + j0 + 1 >= lim) e1 = 0.f;
-              rs += e0 + e1;
-              pk[u] = pack_bf16x2(e0, e1);
+            for (int j = 0; j < 64; ++j) {
+              const float x = (!MK || 64 * h + j < lim) ? __uint_as_float(sr[j]) : -CUDART_INF_F;
+              mxv[j & 7] = fmaxf(mxv[j & 7], x);
             }
-            const uint32_t addr = sPx + h * HALF + row * 128 + ((((uint32_t)c) ^ ((uint32_t)row & 7u)) << 4);
-            st_shared_v4(addr, pk[0], pk[1], pk[2], pk[3]);
           }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_free(grp));
+          const float mx = fmaxf(fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])),
+                                 fmaxf(fmaxf(mxv[4], mxv[5]), fmaxf(mxv[6], mxv[7])));
+          const float mc = fmaxf(m, mx * sl2);
+          need = mc > m + 8.0f;
+          alpha = 1.f;
+          if (need) {
+            alpha = ex2_approx(m - mc);
+            m = mc;
+          }
+          const float mu = (m == -CUDART_INF_F) ? 0.f : m;
+          // The previous PV of this group is complete (it was issued before
+          // this S and tcgen05 work completes in order); the wait is cheap and
+          // makes the P buffer reuse explicit.
+          if (pv_cnt > 0) {
+            mbar_wait(o_done(grp), (pv_cnt - 1) & 1, abort_flag, cap);
+            tc_fence_after();
+          }
+          // pass 2: P = 2^(s*scale*log2e - m) as bf16 pairs written back into
+          // TMEM over columns of S this thread has already read (half h of the
+          // keys lands in columns [32h, 32h+32)); the PV MMA reads it there.
+          float rsv[8];  // eight independent partial row sums
+#pragma unroll
+          for (int u = 0; u < 8; ++u) rsv[u] = 0.f;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t sr[64];
+            tmem_ld32(tS + 64u * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            tmem_ld32(tS + 64u * h + 32u, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+            tmem_wait_ld();
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int u = 0; u < 16; ++u) {
+                const int j0 = 32 * q2 + 2 * u;
+                float e0 = ex2_approx(fmaf(__uint_as_float(sr[j0]), sl2, -mu));
+                float e1 = ex2_approx(fmaf(__uint_as_float(sr[j0 + 1]), sl2, -mu));
+                if (MK && 64 * h + j0 >= lim) e0 = 0.f;
+                if (MK && 64 * h + j0 + 1 >= lim) e1 = 0.f;
+                rsv[(2 * u) & 7] += e0;
+                rsv[(2 * u + 1) & 7] += e1;
+                pk[u] = pack_bf16x2(e0, e1);
+              }
+              tmem_st16(tS + 32u * h + 16u * q2, pk);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free(grp));
+          rs = ((rsv[0] + rsv[1]) + (rsv[2] + rsv[3])) + ((rsv[4] + rsv[5]) + (rsv[6] + rsv[7]));
+        };
+        if (msk) tile(std::true_type{});
+        else tile(std::false_type{});
         l = l * alpha + rs;
         if (n_pv > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
@@ -471,7 +497,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_wait_st();
         }
-        fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full(grp));

@@ -333,16 +333,17 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct BwdLayout {
   int64_t C, Cp;
-  size_t vec_bytes, acc_bytes, total;
+  size_t vec_bytes, total;
 };
 
+// Backward scratch: LSE*log2(e) and D per head in padded rows (two arrays).
 BwdLayout bwd_layout(int64_t N, int32_t P, int32_t Hq, int32_t d) {
+  (void)d;
   BwdLayout L;
   L.C = N / (2 * (int64_t)P);
   L.Cp = (L.C + 127) / 128 * 128;
   L.vec_bytes = align256((size_t)Hq * 2 * P * L.Cp * sizeof(float));
-  L.acc_bytes = align256((size_t)N * Hq * d * sizeof(float));
-  L.total = 2 * L.vec_bytes + L.acc_bytes;
+  L.total = 2 * L.vec_bytes;
   return L;
 }
 }  // namespace
@@ -382,15 +383,14 @@ extern "C" int mmsp_attn_bwd(const void* q, const void* k, const void* v, const 
   char* ws = static_cast<char*>(workspace);
   float* lse2t = reinterpret_cast<float*>(ws);
   float* dt = reinterpret_cast<float*>(ws + Lw.vec_bytes);
-  float* acc = dq_acc_opt ? dq_acc_opt : reinterpret_cast<float*>(ws + 2 * Lw.vec_bytes);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   const int64_t pre_warps = (int64_t)P * 2 * Lw.Cp * Hq;
   int64_t pre_blocks = (pre_warps + 7) / 8;
   if (pre_blocks > 16LL * sms) pre_blocks = 16LL * sms;
-  bwd::bwd_pre_kernel<<<(unsigned)pre_blocks, 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2t, dt, acc, P, Hq,
-      Lw.C, Lw.Cp, 1);
+  bwd::bwd_pre_kernel<<<(unsigned)pre_blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
+                                                             static_cast<const __nv_bfloat16*>(dout), lse, lse2t, dt,
+                                                             P, Hq, Lw.C, Lw.Cp);
   MMSP_CUDA(cudaGetLastError());
 
   bwd::Params p;
@@ -403,31 +403,31 @@ extern "C" int mmsp_attn_bwd(const void* q, const void* k, const void* v, const 
   p.ntiles = (int32_t)(Lw.Cp / 128);
   p.causal = causal;
   p.n_units = 2LL * P * p.ntiles * Hkv;
+  p.n_items = 2LL * P * p.ntiles * Hq;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.scale = scale;
   p.lse2t = lse2t;
   p.dt = dt;
-  p.dq_acc = acc;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dq_acc = dq_acc_opt;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.wait_cap = kWaitCapCycles;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_dev[dev].bwd_attr[1]) {
-      MMSP_CUDA(cudaFuncSetAttribute(bwd::attn_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     bwd::Smem::ALLOC));
+      MMSP_CUDA(cudaFuncSetAttribute(bwd::attn_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     bwd::SmemKV::ALLOC));
+      MMSP_CUDA(cudaFuncSetAttribute(bwd::attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     bwd::SmemQ::ALLOC));
       g_dev[dev].bwd_attr[1] = true;
     }
   }
-  const int64_t grid = p.n_units < sms ? p.n_units : sms;
-  bwd::attn_bwd_kernel<<<(unsigned)grid, bwd::kThreads, bwd::Smem::ALLOC, st>>>(tq, tk, tv, tdo, p);
+  const int64_t grid_kv = p.n_units < sms ? p.n_units : sms;
+  bwd::attn_bwd_dkdv_kernel<<<(unsigned)grid_kv, bwd::kThreads, bwd::SmemKV::ALLOC, st>>>(tq, tk, tv, tdo, p);
   MMSP_CUDA(cudaGetLastError());
-
-  const int64_t n4 = N * Hq * d / 4;
-  int64_t cblocks = (n4 + 255) / 256;
-  if (cblocks > 16LL * sms) cblocks = 16LL * sms;
-  bwd::bwd_dq_convert_kernel<<<(unsigned)cblocks, 256, 0, st>>>(reinterpret_cast<const float4*>(acc),
-                                                                 static_cast<uint2*>(dq), n4);
+  const int64_t grid_q = p.n_items < sms ? p.n_items : sms;
+  bwd::attn_bwd_dq_kernel<<<(unsigned)grid_q, bwd::kThreads, bwd::SmemQ::ALLOC, st>>>(tq, tk, tv, tdo, p);
   MMSP_CUDA(cudaGetLastError());
   return ok();
 }

@@ -55,7 +55,7 @@ def test_noalloc_backward_matches_workspace_backward_twice_in_a_row():
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     m = lib()
-    N, P, hq = 8192, 4, 28
+    N, P, hq = 524288, 64, 28
     assert m.mmsp_bwd_workspace_bytes(N, P, hq, 128) > m.MMSP_NOALLOC_SCRATCH_BYTES
     x = torch.zeros(16, device="cuda", dtype=torch.bfloat16)
     with pytest.raises(m.MmspError) as e:
