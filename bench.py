@@ -253,7 +253,7 @@ class Path:
         self.ws_bytes = m.mmsp_bwd_workspace_bytes(N, P, hq, d)
         self.ws = e(self.ws_bytes, dt=torch.uint8)
         self.scale = 1.0 / math.sqrt(d)
-        self.launches_per_step = 2 + 4 + 1 + 3 + 4
+        self.launches_per_step = 2 + 4 + 1 + 3 + 4  # maps+counts, 4 gathers, fwd, bwd x3, 4 scatters
 
     def step(self, stream, ev=None):
         m, w = self.m, self.w
@@ -268,10 +268,19 @@ class Path:
                         self.ol, m.MMSP_FINALIZE, stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        m.mmsp_attn_bwd(self.ql, self.kl, self.vl, self.ol, self.dol, self.lse, N, P, w.hq, w.hkv, w.d,
-                        self.scale, 1, self.dql, self.dkl, self.dvl, None, self.ws, self.ws_bytes, stream=stream)
+        # the backward's three stages (what mmsp_attn_bwd runs), so that the
+        # dominant dK/dV kernel can be timed on its own
+        m.mmsp_attn_bwd_prepare(self.ol, self.dol, self.lse, N, P, w.hq, w.d, self.ws, self.ws_bytes, stream=stream)
         if ev is not None:
             ev[2].record(stream)
+        m.mmsp_attn_bwd_dkdv(self.ql, self.kl, self.vl, self.dol, N, P, w.hq, w.hkv, w.d, self.scale, 1, self.dkl,
+                             self.dvl, self.ws, self.ws_bytes, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+        m.mmsp_attn_bwd_dq(self.ql, self.kl, self.vl, self.dol, N, P, w.hq, w.hkv, w.d, self.scale, 1, self.dql, None,
+                           self.ws, self.ws_bytes, stream=stream)
+        if ev is not None:
+            ev[4].record(stream)
         for src, dst in ((self.ol, self.o), (self.dql, self.dq), (self.dkl, self.dk), (self.dvl, self.dv)):
             m.mmsp_shard(None, None, N, P, src=src, dst=dst, row_bytes=src[0].numel() * 2, inverse=True,
                          stream=stream)
@@ -303,7 +312,7 @@ def run_gpu(args):
     m.mmsp_device_status(stream)
 
     # ---------------- device-resident timing
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
     sampler = ClockSampler(cvd.split(",")[local] if cvd else local)
@@ -319,7 +328,9 @@ def run_gpu(args):
     m.mmsp_device_status(stream)
     ms_total = t_start.elapsed_time(t_end)
     fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
-    bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    bwd_ms = float(np.mean([e[1].elapsed_time(e[4]) for e in evs]))
+    dkdv_ms = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
+    dq_ms = float(np.mean([e[3].elapsed_time(e[4]) for e in evs]))
     ok = bool(torch.isfinite(path.dq.float()).all()) and bool(torch.isfinite(path.o.float()).all())
 
     # ---------------- end to end through the C ABI with host buffers
@@ -346,16 +357,19 @@ def run_gpu(args):
     m.mmsp_device_status(stream)
 
     # ---------------- max over ranks
-    ms_total, e2e_ms, fwd_ms, bwd_ms = max_over_ranks([ms_total, e2e_ms, fwd_ms, bwd_ms], ws, dev)
+    ms_total, e2e_ms, fwd_ms, bwd_ms, dkdv_ms, dq_ms = max_over_ranks(
+        [ms_total, e2e_ms, fwd_ms, bwd_ms, dkdv_ms, dq_ms], ws, dev)
     ms_step = ms_total / args.steps
     flops = w.fwd_bwd_flops()
     value = job_throughput(flops, ws, ms_step)
     if rank == 0:
         peaks, src = load_peaks()
         peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-        bwd_flops = 2.5 * w.fwd_flops()
-        achieved = bwd_flops / (bwd_ms * 1e-3) / 1e12
-        traffic = profiled_traffic(f"attn_bwd_{w.name}.md", ["attn_bwd.cuh", "ptx.cuh"])
+        # dominant kernel (ncu launch list): the dK/dV kernel; its algorithmic
+        # work is the four GEMM-equivalents S^T, dP^T, dV, dK = 2x forward
+        dkdv_flops = 2.0 * w.fwd_flops()
+        achieved = dkdv_flops / (dkdv_ms * 1e-3) / 1e12
+        traffic = profiled_traffic(f"attn_bwd_dkdv_{w.name}.md", ["attn_bwd.cuh", "ptx.cuh"])
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -365,10 +379,14 @@ def run_gpu(args):
             "frac_of_bf16_peak": {"fwd": w.fwd_flops() / (fwd_ms * 1e-3) / 1e12 / peak,
                                   "fwd_bwd": value / ws / peak, "peak_tflops": peak,
                                   "peak_kind": f"bf16_tflops_sustained ({src})"},
-            "roofline": {"kernel": "attn_bwd (mmsp_attn_bwd: D preprocess + tcgen05 main + dQ convert)",
+            "roofline": {"kernel": "attn_bwd_dkdv_kernel (mmsp_attn_bwd_dkdv)",
                          "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
+                         "algorithmic_flops_per_launch": dkdv_flops, "launch_ms": dkdv_ms,
                          "peak_source": f"MEASURED_PEAKS.json bf16_tflops_sustained ({src})"},
+            "bwd_tflops": 2.5 * w.fwd_flops() / (bwd_ms * 1e-3) / 1e12,
+            "kernel_ms": {"attn_fwd": fwd_ms, "attn_bwd_dkdv": dkdv_ms, "attn_bwd_dq": dq_ms,
+                          "bwd_total": bwd_ms},
             "e2e": {"value": flops * ws / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": path.launches_per_step * args.steps,

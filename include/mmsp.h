@@ -173,6 +173,32 @@ int mmsp_attn_bwd(const void* q, const void* k, const void* v,
                   void* dq, void* dk, void* dv, float* dq_acc_opt,
                   void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * The three stages mmsp_attn_bwd runs, in this order, exported for callers
+ * that want them separately (to time or overlap them, or to skip dQ):
+ *   mmsp_attn_bwd_prepare -- D = rowsum(dO * O) and LSE*log2(e) per head
+ *                            into `workspace` (one bandwidth-bound kernel);
+ *   mmsp_attn_bwd_dkdv    -- dK, dV: key-owner tcgen05 kernel, one kv head
+ *                            x 128 keys per work unit;
+ *   mmsp_attn_bwd_dq      -- dQ (bf16, plus fp32 into dq_acc_opt if
+ *                            non-NULL): query-owner tcgen05 kernel, one
+ *                            query head x 128 rows per work item.
+ * dkdv and dq read the prepared workspace and may run in either order. The
+ * arguments mean what they mean for mmsp_attn_bwd; each call validates its
+ * own and returns MMSP_EINVAL/MMSP_EUNSUPPORTED without launching.
+ */
+int mmsp_attn_bwd_prepare(const void* o, const void* dout, const float* lse,
+                          int64_t N, int32_t P, int32_t Hq, int32_t d,
+                          void* workspace, size_t workspace_bytes, void* stream);
+int mmsp_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout,
+                       int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d,
+                       float scale, int32_t causal, void* dk, void* dv,
+                       const void* workspace, size_t workspace_bytes, void* stream);
+int mmsp_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dout,
+                     int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d,
+                     float scale, int32_t causal, void* dq, float* dq_acc_opt,
+                     const void* workspace, size_t workspace_bytes, void* stream);
+
 /* Scratch bytes mmsp_attn_bwd needs for these sizes (0 on invalid sizes). */
 size_t mmsp_bwd_workspace_bytes(int64_t N, int32_t P, int32_t Hq, int32_t d);
 

@@ -15,6 +15,9 @@ from ._binding import (  # noqa: F401
     lib_path,
     mmsp_attn_bwd,
     mmsp_attn_bwd_noalloc,
+    mmsp_attn_bwd_prepare,
+    mmsp_attn_bwd_dkdv,
+    mmsp_attn_bwd_dq,
     MMSP_NOALLOC_SCRATCH_BYTES,
     mmsp_attn_fwd,
     mmsp_bwd_workspace_bytes,

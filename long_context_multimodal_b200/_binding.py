@@ -47,6 +47,12 @@ _SIGS = {
     "mmsp_attn_bwd": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32,
                        c_int32, c_int32, c_float, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                        c_size_t, c_void_p], c_int32),
+    "mmsp_attn_bwd_prepare": ([c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32, c_int32, c_void_p, c_size_t,
+                               c_void_p], c_int32),
+    "mmsp_attn_bwd_dkdv": ([c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32, c_int32, c_int32,
+                            c_float, c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p], c_int32),
+    "mmsp_attn_bwd_dq": ([c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32, c_int32, c_int32,
+                          c_float, c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p], c_int32),
     "mmsp_bwd_workspace_bytes": ([c_int64, c_int32, c_int32, c_int32], c_size_t),
     "mmsp_attn_bwd_noalloc": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32,
                                c_int32, c_int32, c_int32, c_float, c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -142,6 +148,28 @@ def mmsp_attn_bwd(q, k, v, o, dout, lse, N, P, Hq, Hkv, d, scale, causal, dq, dk
                             int(Hkv), int(d), float(scale), int(causal), _ptr(dq), _ptr(dk), _ptr(dv),
                             _ptr(dq_acc_opt), _ptr(workspace), int(workspace_bytes), _stream(stream))
     return _check("mmsp_attn_bwd", rc)
+
+
+def mmsp_attn_bwd_prepare(o, dout, lse, N, P, Hq, d, workspace, workspace_bytes, stream=None):
+    rc = _lib.mmsp_attn_bwd_prepare(_ptr(o), _ptr(dout), _ptr(lse), int(N), int(P), int(Hq), int(d), _ptr(workspace),
+                                    int(workspace_bytes), _stream(stream))
+    return _check("mmsp_attn_bwd_prepare", rc)
+
+
+def mmsp_attn_bwd_dkdv(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, dk, dv, workspace, workspace_bytes,
+                       stream=None):
+    rc = _lib.mmsp_attn_bwd_dkdv(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), int(N), int(P), int(Hq), int(Hkv), int(d),
+                                 float(scale), int(causal), _ptr(dk), _ptr(dv), _ptr(workspace),
+                                 int(workspace_bytes), _stream(stream))
+    return _check("mmsp_attn_bwd_dkdv", rc)
+
+
+def mmsp_attn_bwd_dq(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, dq, dq_acc_opt, workspace, workspace_bytes,
+                     stream=None):
+    rc = _lib.mmsp_attn_bwd_dq(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), int(N), int(P), int(Hq), int(Hkv), int(d),
+                               float(scale), int(causal), _ptr(dq), _ptr(dq_acc_opt), _ptr(workspace),
+                               int(workspace_bytes), _stream(stream))
+    return _check("mmsp_attn_bwd_dq", rc)
 
 
 def mmsp_attn_bwd_noalloc(q, k, v, o, dout, lse, N, P, Hq, Hkv, d, scale, causal, dq, dk, dv, dq_acc_opt,

@@ -10,6 +10,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 
 #include "mmsp.h"
@@ -353,83 +354,152 @@ extern "C" size_t mmsp_bwd_workspace_bytes(int64_t N, int32_t P, int32_t Hq, int
   return bwd_layout(N, P, Hq, d).total;
 }
 
-extern "C" int mmsp_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                             const float* lse, int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d, float scale,
-                             int32_t causal, void* dq, void* dk, void* dv, float* dq_acc_opt, void* workspace,
-                             size_t workspace_bytes, void* stream) {
+namespace {
+// Shared checks of the backward stages (sizes, scale, workspace).
+int bwd_check(int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d, float scale, int32_t causal,
+              const void* workspace, size_t workspace_bytes) {
   int rc = check_common(N, P);
   if (rc) return rc;
   if ((rc = check_heads(Hq, Hkv, d))) return rc;
-  if (d != 128) return fail(MMSP_EUNSUPPORTED, "mmsp_attn_bwd supports d = 128 (got %d)", d);
+  if (d != 128) return fail(MMSP_EUNSUPPORTED, "the backward supports d = 128 (got %d)", d);
   if (!(scale > 0.f) || !std::isfinite(scale)) return fail(MMSP_EINVAL, "scale must be finite and > 0");
   if (causal != 0 && causal != 1) return fail(MMSP_EINVAL, "causal must be 0 or 1");
-  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv)
-    return fail(MMSP_EINVAL, "q, k, v, o, dout, lse, dq, dk, dv must be non-NULL");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
-      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (dq_acc_opt && !aligned16(dq_acc_opt)))
-    return fail(MMSP_EINVAL, "all tensors must be 16-byte aligned");
-  if (N == 0) return ok();
+  if (N == 0) return MMSP_OK;
   const BwdLayout Lw = bwd_layout(N, P, Hq, d);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return fail(MMSP_EINVAL, "workspace must be non-NULL and 256-byte aligned");
   if (workspace_bytes < Lw.total)
     return fail(MMSP_EINVAL, "workspace too small: %zu < %zu bytes", workspace_bytes, Lw.total);
-  int dev, sms;
-  if ((rc = current_device(&dev)) || (rc = device_sms(dev, &sms)) || (rc = get_encode())) return rc;
-  CUtensorMap tq, tk, tv, tdo;
-  if ((rc = tmap_rows_heads(&tq, q, N, Hq, d)) || (rc = tmap_rows_heads(&tk, k, N, Hkv, d)) ||
-      (rc = tmap_rows_heads(&tv, v, N, Hkv, d)) || (rc = tmap_rows_heads(&tdo, dout, N, Hq, d)))
-    return rc;
-  char* ws = static_cast<char*>(workspace);
-  float* lse2t = reinterpret_cast<float*>(ws);
-  float* dt = reinterpret_cast<float*>(ws + Lw.vec_bytes);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return MMSP_OK;
+}
 
+bool all_aligned16(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (p && !aligned16(p)) return false;
+  return true;
+}
+
+// Parameters and tensor maps of the two tcgen05 backward kernels.
+int bwd_setup(const void* q, const void* k, const void* v, const void* dout, int64_t N, int32_t P, int32_t Hq,
+              int32_t Hkv, int32_t d, float scale, int32_t causal, const void* workspace, bwd::Params* p,
+              CUtensorMap* tq, CUtensorMap* tk, CUtensorMap* tv, CUtensorMap* tdo, int* sms) {
+  int dev, rc;
+  if ((rc = current_device(&dev)) || (rc = device_sms(dev, sms)) || (rc = get_encode())) return rc;
+  if ((rc = tmap_rows_heads(tq, q, N, Hq, d)) || (rc = tmap_rows_heads(tk, k, N, Hkv, d)) ||
+      (rc = tmap_rows_heads(tv, v, N, Hkv, d)) || (rc = tmap_rows_heads(tdo, dout, N, Hq, d)))
+    return rc;
+  const BwdLayout Lw = bwd_layout(N, P, Hq, d);
+  const char* ws = static_cast<const char*>(workspace);
+  *p = bwd::Params{};
+  p->P = P;
+  p->Hq = Hq;
+  p->Hkv = Hkv;
+  p->G = Hq / Hkv;
+  p->C = Lw.C;
+  p->Cp = Lw.Cp;
+  p->ntiles = (int32_t)(Lw.Cp / 128);
+  p->causal = causal;
+  p->n_units = 2LL * P * p->ntiles * Hkv;
+  p->n_items = 2LL * P * p->ntiles * Hq;
+  p->scale_log2 = scale * 1.4426950408889634f;
+  p->scale = scale;
+  p->lse2t = reinterpret_cast<const float*>(ws);
+  p->dt = reinterpret_cast<const float*>(ws + Lw.vec_bytes);
+  p->wait_cap = kWaitCapCycles;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_dev[dev].bwd_attr[1]) {
+    MMSP_CUDA(cudaFuncSetAttribute(bwd::attn_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   bwd::SmemKV::ALLOC));
+    MMSP_CUDA(cudaFuncSetAttribute(bwd::attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   bwd::SmemQ::ALLOC));
+    g_dev[dev].bwd_attr[1] = true;
+  }
+  return MMSP_OK;
+}
+}  // namespace
+
+extern "C" int mmsp_attn_bwd_prepare(const void* o, const void* dout, const float* lse, int64_t N, int32_t P,
+                                     int32_t Hq, int32_t d, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = bwd_check(N, P, Hq, 1, d, 1.f, 1, workspace, workspace_bytes);
+  if (rc) return rc;
+  if (!o || !dout || !lse) return fail(MMSP_EINVAL, "o, dout and lse must be non-NULL");
+  if (!all_aligned16({o, dout, lse})) return fail(MMSP_EINVAL, "all tensors must be 16-byte aligned");
+  if (N == 0) return ok();
+  int dev, sms;
+  if ((rc = current_device(&dev)) || (rc = device_sms(dev, &sms))) return rc;
+  const BwdLayout Lw = bwd_layout(N, P, Hq, d);
+  char* ws = static_cast<char*>(workspace);
   const int64_t pre_warps = (int64_t)P * 2 * Lw.Cp * Hq;
   int64_t pre_blocks = (pre_warps + 7) / 8;
   if (pre_blocks > 16LL * sms) pre_blocks = 16LL * sms;
-  bwd::bwd_pre_kernel<<<(unsigned)pre_blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
-                                                             static_cast<const __nv_bfloat16*>(dout), lse, lse2t, dt,
-                                                             P, Hq, Lw.C, Lw.Cp);
-  MMSP_CUDA(cudaGetLastError());
-
-  bwd::Params p;
-  p.P = P;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.G = Hq / Hkv;
-  p.C = Lw.C;
-  p.Cp = Lw.Cp;
-  p.ntiles = (int32_t)(Lw.Cp / 128);
-  p.causal = causal;
-  p.n_units = 2LL * P * p.ntiles * Hkv;
-  p.n_items = 2LL * P * p.ntiles * Hq;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.scale = scale;
-  p.lse2t = lse2t;
-  p.dt = dt;
-  p.dq = static_cast<__nv_bfloat16*>(dq);
-  p.dq_acc = dq_acc_opt;
-  p.dk = static_cast<__nv_bfloat16*>(dk);
-  p.dv = static_cast<__nv_bfloat16*>(dv);
-  p.wait_cap = kWaitCapCycles;
-  {
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_dev[dev].bwd_attr[1]) {
-      MMSP_CUDA(cudaFuncSetAttribute(bwd::attn_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     bwd::SmemKV::ALLOC));
-      MMSP_CUDA(cudaFuncSetAttribute(bwd::attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     bwd::SmemQ::ALLOC));
-      g_dev[dev].bwd_attr[1] = true;
-    }
-  }
-  const int64_t grid_kv = p.n_units < sms ? p.n_units : sms;
-  bwd::attn_bwd_dkdv_kernel<<<(unsigned)grid_kv, bwd::kThreads, bwd::SmemKV::ALLOC, st>>>(tq, tk, tv, tdo, p);
-  MMSP_CUDA(cudaGetLastError());
-  const int64_t grid_q = p.n_items < sms ? p.n_items : sms;
-  bwd::attn_bwd_dq_kernel<<<(unsigned)grid_q, bwd::kThreads, bwd::SmemQ::ALLOC, st>>>(tq, tk, tv, tdo, p);
+  bwd::bwd_pre_kernel<<<(unsigned)pre_blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse,
+      reinterpret_cast<float*>(ws), reinterpret_cast<float*>(ws + Lw.vec_bytes), P, Hq, Lw.C, Lw.Cp);
   MMSP_CUDA(cudaGetLastError());
   return ok();
+}
+
+extern "C" int mmsp_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout, int64_t N,
+                                  int32_t P, int32_t Hq, int32_t Hkv, int32_t d, float scale, int32_t causal,
+                                  void* dk, void* dv, const void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = bwd_check(N, P, Hq, Hkv, d, scale, causal, workspace, workspace_bytes);
+  if (rc) return rc;
+  if (!q || !k || !v || !dout || !dk || !dv) return fail(MMSP_EINVAL, "q, k, v, dout, dk, dv must be non-NULL");
+  if (!all_aligned16({q, k, v, dout, dk, dv})) return fail(MMSP_EINVAL, "all tensors must be 16-byte aligned");
+  if (N == 0) return ok();
+  bwd::Params p;
+  CUtensorMap tq, tk, tv, tdo;
+  int sms;
+  if ((rc = bwd_setup(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, workspace, &p, &tq, &tk, &tv, &tdo, &sms)))
+    return rc;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  const int64_t grid = p.n_units < sms ? p.n_units : sms;
+  bwd::attn_bwd_dkdv_kernel<<<(unsigned)grid, bwd::kThreads, bwd::SmemKV::ALLOC, static_cast<cudaStream_t>(stream)>>>(
+      tq, tk, tv, tdo, p);
+  MMSP_CUDA(cudaGetLastError());
+  return ok();
+}
+
+extern "C" int mmsp_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dout, int64_t N, int32_t P,
+                                int32_t Hq, int32_t Hkv, int32_t d, float scale, int32_t causal, void* dq,
+                                float* dq_acc_opt, const void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = bwd_check(N, P, Hq, Hkv, d, scale, causal, workspace, workspace_bytes);
+  if (rc) return rc;
+  if (!q || !k || !v || !dout || !dq) return fail(MMSP_EINVAL, "q, k, v, dout, dq must be non-NULL");
+  if (!all_aligned16({q, k, v, dout, dq, dq_acc_opt})) return fail(MMSP_EINVAL, "all tensors must be 16-byte aligned");
+  if (N == 0) return ok();
+  bwd::Params p;
+  CUtensorMap tq, tk, tv, tdo;
+  int sms;
+  if ((rc = bwd_setup(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, workspace, &p, &tq, &tk, &tv, &tdo, &sms)))
+    return rc;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dq_acc = dq_acc_opt;
+  const int64_t grid = p.n_items < sms ? p.n_items : sms;
+  bwd::attn_bwd_dq_kernel<<<(unsigned)grid, bwd::kThreads, bwd::SmemQ::ALLOC, static_cast<cudaStream_t>(stream)>>>(
+      tq, tk, tv, tdo, p);
+  MMSP_CUDA(cudaGetLastError());
+  return ok();
+}
+
+extern "C" int mmsp_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                             const float* lse, int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d, float scale,
+                             int32_t causal, void* dq, void* dk, void* dv, float* dq_acc_opt, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  int rc = bwd_check(N, P, Hq, Hkv, d, scale, causal, workspace, workspace_bytes);
+  if (rc) return rc;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv)
+    return fail(MMSP_EINVAL, "q, k, v, o, dout, lse, dq, dk, dv must be non-NULL");
+  if (!all_aligned16({q, k, v, o, dout, lse, dq, dk, dv, dq_acc_opt}))
+    return fail(MMSP_EINVAL, "all tensors must be 16-byte aligned");
+  if (N == 0) return ok();
+  if ((rc = mmsp_attn_bwd_prepare(o, dout, lse, N, P, Hq, d, workspace, workspace_bytes, stream))) return rc;
+  if ((rc = mmsp_attn_bwd_dkdv(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, dk, dv, workspace, workspace_bytes,
+                               stream)))
+    return rc;
+  return mmsp_attn_bwd_dq(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, dq, dq_acc_opt, workspace, workspace_bytes,
+                          stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -78,6 +78,11 @@ def test_merge_and_bwd_reject_bad_arguments():
     _einval(m.mmsp_lse_merge, p + 4, p, p, p, p, p, 10, 2, 64)
     _einval(m.mmsp_lse_merge, p, p, p, p, p, p, -1, 2, 64)
     _einval(m.mmsp_selftest_bounded_wait, 0)
+    # backward stages validate their own arguments
+    _einval(m.mmsp_attn_bwd_prepare, p, p, p, 4096, 4, 28, 128, None, 0)
+    _einval(m.mmsp_attn_bwd_dkdv, p, p, p, p, 4096, 4, 28, 5, 128, 0.1, 1, p, p, p, 1 << 30)
+    _einval(m.mmsp_attn_bwd_dq, p, p, p, p, 4095, 4, 28, 4, 128, 0.1, 1, p, None, p, 1 << 30)
+    _einval(m.mmsp_attn_bwd_dq, p, p, p, p, 4096, 4, 28, 4, 128, 0.1, 1, p + 4, None, p, 1 << 30)
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):

@@ -120,3 +120,24 @@ def test_n512k_sampled_gradients():
 
 def test_n1m_sampled_gradients():
     _full_size("n1m", 192, 64)
+
+
+def test_backward_stages_match_the_single_call():
+    """prepare + dQ + dK/dV called separately (dQ first) give what
+    mmsp_attn_bwd gives."""
+    m = lib()
+    N, P, hq, hkv, d = 1200, 3, 4, 2, 128
+    _, q, k, v, do = inputs(N, hq, hkv, d, seed=5, with_dout=True)
+    ql, kl, vl, dol = (shard_rows(x, N, P) for x in (q, k, v, do))
+    _, lse, o = run_forward(ql, kl, vl, P)
+    dq, dk, dv, _ = run_backward(ql, kl, vl, o, dol, lse, P)
+    wsb = m.mmsp_bwd_workspace_bytes(N, P, hq, d)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    dq2, dk2, dv2 = (torch.full_like(x, float("nan")) for x in (ql, kl, vl))
+    sc = 1 / math.sqrt(d)
+    m.mmsp_attn_bwd_prepare(o, dol, lse, N, P, hq, d, ws, wsb)
+    m.mmsp_attn_bwd_dq(ql, kl, vl, dol, N, P, hq, hkv, d, sc, 1, dq2, None, ws, wsb)
+    m.mmsp_attn_bwd_dkdv(ql, kl, vl, dol, N, P, hq, hkv, d, sc, 1, dk2, dv2, ws, wsb)
+    m.mmsp_device_status()
+    for a, b in ((dq, dq2), (dk, dk2), (dv, dv2)):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
