@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issuer
     // Once P^T_v (TMEM) and dS^T_v (smem) are ready: dV += P^T_v dO_v,
-    // S^T_{v+1} (over P^T_v, after dV read it), dP^T_{v+1}, dK += dS^T_v Q_v.
+    // S^T_{v+1} (over P^T_v, after dV read it), dK += dS^T_v Q_v, dP^T_{v+1}.
     const uint32_t leader = lane == 0 ? 1u : 0u;
     constexpr uint32_t idKQ = idesc_bf16_f32(BM, BN, 0, 0);   // S^T, dP^T
     constexpr uint32_t idGrad = idesc_bf16_f32(BM, D, 0, 1);  // dV, dK: B MN-major
@@ -360,10 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         (kk > 0 || !first) ? 1u : 0u);
         mma_commit_w(leader, do_empty(st));
         has = it.next();
-        if (has) {
-          issue_s(vis + 1);
-          issue_dp(vis + 1);  // the dP^T region was read before p_full
-        }
+        if (has) issue_s(vis + 1);
         // dK += dS^T Q
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
@@ -374,6 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit_w(leader, q_empty(st));
         mma_commit_w(leader, dst_free);
+        if (has) issue_dp(vis + 1);
         ++vis;
         first = false;
       }

@@ -471,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (MK && 64 * h + j0 + 1 >= lim) e1 = 0.f;
                 rsv[(2 * u) & 7] += e0;
                 rsv[(2 * u + 1) & 7] += e1;
-                pk[u] = pack_bf16x2(e0, e1);
+                pk[u] = pack_bf16x2_alu(e0, e1);
               }
               tmem_st16(tS + 32u * h + 16u * q2, pk);
             }

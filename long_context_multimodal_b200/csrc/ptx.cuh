@@ -265,6 +265,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Two floats to a bf16 pair (lo in the low half), rounded to nearest with
+// ties away from zero, on the integer pipe: add half an ulp of bf16 to the
+// bit pattern and keep the high halves. For finite values; used for the
+// softmax probabilities and dS, where ties are vanishingly rare.
+__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
+  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
