@@ -51,19 +51,30 @@ def _f64(x):
     return np.asarray(x, dtype=np.float64)
 
 
-def _rows_forward(qr, rows, K, V, scale):
+def _visible(jmax, rows, lo):
+    """[R, jmax] mask: key j visible to row i iff lo_i <= j <= i (lo_i = 0
+    without documents)."""
+    rows_t = torch.as_tensor(np.asarray(rows, np.int64))
+    j = torch.arange(jmax)[None, :]
+    vis = j <= rows_t[:, None]
+    if lo is not None:
+        vis &= j >= torch.as_tensor(np.asarray(lo, np.int64))[:, None]
+    return vis
+
+
+def _rows_forward(qr, rows, K, V, scale, lo=None):
     """O and LSE for query vectors qr [R,d] at global positions rows [R]
-    against keys K[:i+1], V[:i+1] (one head). Plain formula in fp64 torch
-    CPU ops (multi-threaded; same arithmetic as numpy)."""
+    against keys K[:i+1], V[:i+1] (one head); with `lo`, only keys
+    j >= lo_i of the row's own document. Plain formula in fp64 torch CPU ops
+    (multi-threaded; same arithmetic as numpy)."""
     R = len(rows)
     d = V.shape[1]
     if R == 0:
         return np.zeros((R, d)), np.full(R, NEG_INF)
     jmax = int(np.max(rows)) + 1
     qr, K, V = _t(qr), _t(K[:jmax]), _t(V[:jmax])
-    rows_t = torch.as_tensor(np.asarray(rows, np.int64))
     s = (qr @ K.T) * scale                                       # [R, jmax]
-    visible = torch.arange(jmax)[None, :] <= rows_t[:, None]
+    visible = _visible(jmax, rows, lo)
     s = s.masked_fill(~visible, NEG_INF)
     m = s.max(dim=1).values
     lse = m + torch.log(torch.exp(s - m[:, None]).sum(dim=1))
@@ -72,8 +83,12 @@ def _rows_forward(qr, rows, K, V, scale):
     return O.numpy(), lse.numpy()
 
 
-def causal_attention(q, k, v, scale=None, block: int = 512):
-    """Whole-sequence forward. Returns (O [N,Hq,d], LSE [N,Hq]) in fp64."""
+def causal_attention(q, k, v, scale=None, block: int = 512, doc_start=None):
+    """Whole-sequence forward. Returns (O [N,Hq,d], LSE [N,Hq]) in fp64.
+
+    doc_start (optional, [N] ints, global order): first position of each
+    token's document in a packed sequence; key j is then visible to query i
+    iff doc_start[i] <= j <= i (attention reset at document boundaries)."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     N, hq, d = q.shape
     hkv = k.shape[1]
@@ -85,13 +100,14 @@ def causal_attention(q, k, v, scale=None, block: int = 512):
         kh = kv_head(h, hq, hkv)
         for i0 in range(0, N, block):
             rows = np.arange(i0, min(N, i0 + block))
-            o, l = _rows_forward(q[rows, h], rows, k[:, kh], v[:, kh], scale)
+            lo = None if doc_start is None else np.asarray(doc_start)[rows]
+            o, l = _rows_forward(q[rows, h], rows, k[:, kh], v[:, kh], scale, lo)
             O[rows, h] = o
             LSE[rows, h] = l
     return O, LSE
 
 
-def attention_rows(q_rows, k, v, rows, scale=None, block: int = 64):
+def attention_rows(q_rows, k, v, rows, scale=None, block: int = 64, doc_start=None):
     """Forward for selected global rows only.
 
     q_rows [R,Hq,d] holds the query vectors of global positions `rows` (the
@@ -116,20 +132,20 @@ def attention_rows(q_rows, k, v, rows, scale=None, block: int = 64):
                 continue
             for b0 in range(0, R, block):
                 sel = np.arange(b0, min(R, b0 + block))
-                o, l = _rows_forward(q_rows[sel, h], rows[sel], K, V, scale)
+                lo = None if doc_start is None else np.asarray(doc_start)[rows[sel]]
+                o, l = _rows_forward(q_rows[sel, h], rows[sel], K, V, scale, lo)
                 O[sel, h] = o
                 LSE[sel, h] = l
     return O, LSE
 
 
-def _rows_backward(qr, dor, rows, K, V, scale):
+def _rows_backward(qr, dor, rows, K, V, scale, lo=None):
     """For one head and query rows: (O, LSE, D, dQ rows, P, dS) restricted to
     keys [0, max(rows)]; P and dS are [R, jmax]. fp64 torch CPU ops."""
     jmax = int(np.max(rows)) + 1
     qr, dor, K, V = _t(qr), _t(dor), _t(K[:jmax]), _t(V[:jmax])
-    rows_t = torch.as_tensor(np.asarray(rows, np.int64))
     s = (qr @ K.T) * scale
-    visible = torch.arange(jmax)[None, :] <= rows_t[:, None]
+    visible = _visible(jmax, rows, lo)
     s = s.masked_fill(~visible, NEG_INF)
     m = s.max(dim=1).values
     lse = m + torch.log(torch.exp(s - m[:, None]).sum(dim=1))
@@ -142,8 +158,9 @@ def _rows_backward(qr, dor, rows, K, V, scale):
     return o.numpy(), lse.numpy(), D.numpy(), dq.numpy(), p.numpy(), ds.numpy()
 
 
-def causal_attention_bwd(q, k, v, do, scale=None, block: int = 512):
-    """Whole-sequence backward of the definition.
+def causal_attention_bwd(q, k, v, do, scale=None, block: int = 512, doc_start=None):
+    """Whole-sequence backward of the definition (doc_start as in
+    causal_attention).
 
     Returns dict with O, LSE, D [N,Hq], dQ [N,Hq,d], dK, dV [N,Hkv,d] (fp64).
     """
@@ -162,8 +179,9 @@ def causal_attention_bwd(q, k, v, do, scale=None, block: int = 512):
         kh = kv_head(h, hq, hkv)
         for i0 in range(0, N, block):
             rows = np.arange(i0, min(N, i0 + block))
+            lo = None if doc_start is None else np.asarray(doc_start)[rows]
             o, lse, D, dq, p, ds = _rows_backward(q[rows, h], do[rows, h], rows,
-                                                  k[:, kh], v[:, kh], scale)
+                                                  k[:, kh], v[:, kh], scale, lo)
             jmax = p.shape[1]
             O[rows, h] = o
             LSE[rows, h] = lse

@@ -110,3 +110,46 @@ def test_rows_equal_full():
 def test_gqa_mapping_is_contiguous_groups():
     assert [A.kv_head(h, 28, 4) for h in range(28)] == [h // 7 for h in range(28)]
     assert [A.kv_head(h, 4, 4) for h in range(4)] == [0, 1, 2, 3]
+
+
+def _doc_start(lengths):
+    out = []
+    pos = 0
+    for L in lengths:
+        out += [pos] * L
+        pos += L
+    return np.asarray(out, np.int64)
+
+
+def test_document_mask_equals_separate_documents():
+    """Packed sequence with attention reset at document boundaries = plain
+    causal attention of each document on its own (brute force)."""
+    rng = np.random.default_rng(12)
+    lengths = [7, 1, 30, 12, 50]
+    N = sum(lengths)
+    q = rng.standard_normal((N, 4, 8))
+    k = rng.standard_normal((N, 2, 8)) * 2
+    v = rng.standard_normal((N, 2, 8))
+    ds = _doc_start(lengths)
+    O, L = A.causal_attention(q, k, v, block=16, doc_start=ds)
+    pos = 0
+    for Ln in lengths:
+        sl = slice(pos, pos + Ln)
+        Od, Ld = A.causal_attention(q[sl], k[sl], v[sl])
+        np.testing.assert_allclose(O[sl], Od, atol=1e-12)
+        np.testing.assert_allclose(L[sl], Ld, atol=1e-12)
+        pos += Ln
+    # sampled rows agree with the whole-sequence version
+    rows = np.array([0, 6, 7, 8, 37, 38, 99])
+    Or, Lr = A.attention_rows(q[rows], k, v, rows, block=3, doc_start=ds)
+    np.testing.assert_allclose(Or, O[rows], atol=1e-12)
+    np.testing.assert_allclose(Lr, L[rows], atol=1e-12)
+
+
+def test_single_document_is_plain_causal():
+    rng = np.random.default_rng(13)
+    q, k, v = rng.standard_normal((3, 40, 2, 8))
+    O, L = A.causal_attention(q, k, v, doc_start=np.zeros(40, np.int64))
+    O2, L2 = A.causal_attention(q, k, v)
+    np.testing.assert_array_equal(O, O2)
+    np.testing.assert_array_equal(L, L2)

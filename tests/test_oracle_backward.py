@@ -83,3 +83,18 @@ def test_rows_and_keys_variants_equal_full():
     kk = A.attention_bwd_keys(q[60:], k, v, do[60:], keys, block=7)
     np.testing.assert_allclose(kk["dK"], g["dK"][keys], atol=1e-12)
     np.testing.assert_allclose(kk["dV"], g["dV"][keys], atol=1e-12)
+
+
+def test_document_mask_backward_equals_separate_documents():
+    lengths = [9, 20, 1, 14]
+    N = sum(lengths)
+    q, k, v, do = _inputs(N, 4, 2, 8, 21)
+    ds = np.concatenate([[sum(lengths[:i])] * L for i, L in enumerate(lengths)]).astype(np.int64)
+    g = A.causal_attention_bwd(q, k, v, do, block=8, doc_start=ds)
+    pos = 0
+    for L in lengths:
+        sl = slice(pos, pos + L)
+        gd = A.causal_attention_bwd(q[sl], k[sl], v[sl], do[sl])
+        for name in ("O", "dQ", "dK", "dV"):
+            np.testing.assert_allclose(g[name][sl], gd[name], atol=1e-12)
+        pos += L

@@ -18,7 +18,7 @@ def test_interleaved_gqa_mapping_is_caught(monkeypatch):
 def test_wrong_scale_is_caught(monkeypatch):
     real = A._rows_forward
     monkeypatch.setattr(A, "_rows_forward",
-                        lambda qr, rows, K, V, scale: real(qr, rows, K, V, scale * 2.0))
+                        lambda qr, rows, K, V, scale, lo=None: real(qr, rows, K, V, scale * 2.0, lo))
     with pytest.raises(AssertionError):
         TA.test_matches_torch_sdpa_fp64(37, 4, 4, 16)
 
