@@ -118,6 +118,14 @@ int mmsp_shard(const int32_t* seg_len, const uint8_t* seg_kind, int32_t n_seg,
  *   o_out              DEVICE bf16 [P][2C][Hq][d]: written (round to nearest
  *                      even) when flags has MMSP_FINALIZE; else may be NULL.
  *   flags              MMSP_ACCUMULATE | MMSP_FINALIZE.
+ *   doc_start          DEVICE int32 [N] in GLOBAL order, or NULL: the first
+ *                      position of each token's document when several
+ *                      documents are packed into one sequence (see
+ *                      mmsp_doc_starts). Key j is then visible to query i
+ *                      iff doc_start[i] <= j <= i. Needs causal == 1; must
+ *                      be non-decreasing with doc_start[i] <= i (not
+ *                      checked: other values give unspecified, finite-time
+ *                      results). NULL: one document.
  * Without MMSP_ACCUMULATE the state starts empty (LSE -inf, O 0).
  * All pointers 16-byte aligned. fp32 accumulation; tcgen05 tensor cores.
  */
@@ -126,7 +134,28 @@ int mmsp_attn_fwd(const void* q, const void* k, const void* v,
                   float scale, int32_t causal,
                   int32_t step_begin, int32_t step_end,
                   float* o_acc, float* lse, void* o_out,
-                  uint32_t flags, void* stream);
+                  uint32_t flags, const int32_t* doc_start, void* stream);
+
+/*
+ * mmsp_doc_starts -- doc_start[g] for a packed sequence given as document
+ * lengths: the position where the document holding global position g
+ * begins.
+ *
+ * Source: "LongVILA Guide" (aifetchly), section "Critical Operational Best
+ * Practices" (dynamic sequence packing: several shorter videos in one long
+ * buffer with the attention mask reset between them) and the Stage 3
+ * paragraph of the three-stage curriculum (variable-length video segments
+ * packed into one long batch). Reading: attention is causal inside each
+ * document and nothing crosses a document boundary.
+ *
+ *   doc_len            HOST int32[n_doc], each >= 1, summing to N;
+ *                      1 <= n_doc <= MMSP_MAX_SEGMENTS (ignored when N == 0).
+ *   N                  total tokens, 0 <= N < 2^31.
+ *   doc_start          DEVICE int32[N] (output), 4-byte aligned.
+ * Bit-exact integer work; returns MMSP_EINVAL without launching on bad input.
+ */
+int mmsp_doc_starts(const int32_t* doc_len, int32_t n_doc, int64_t N,
+                    int32_t* doc_start, void* stream);
 
 /*
  * mmsp_lse_merge -- combine two partial attention results over disjoint key
@@ -164,14 +193,17 @@ int mmsp_lse_merge(const float* o_a, const float* lse_a,
  *                      bytes (per-head LSE*log2(e) and D rows, about 8*Hq
  *                      bytes per token), 256-byte aligned; contents need not
  *                      be zeroed.
- *   d == 128 or 64; other constraints as mmsp_attn_fwd.
+ *   doc_start          as in mmsp_attn_fwd (the same array the forward used).
+ *   d == 128 (MMSP_EUNSUPPORTED otherwise); other constraints as
+ *   mmsp_attn_fwd.
  */
 int mmsp_attn_bwd(const void* q, const void* k, const void* v,
                   const void* o, const void* dout, const float* lse,
                   int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d,
                   float scale, int32_t causal,
                   void* dq, void* dk, void* dv, float* dq_acc_opt,
-                  void* workspace, size_t workspace_bytes, void* stream);
+                  void* workspace, size_t workspace_bytes,
+                  const int32_t* doc_start, void* stream);
 
 /*
  * The three stages mmsp_attn_bwd runs, in this order, exported for callers
@@ -193,11 +225,13 @@ int mmsp_attn_bwd_prepare(const void* o, const void* dout, const float* lse,
 int mmsp_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout,
                        int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d,
                        float scale, int32_t causal, void* dk, void* dv,
-                       const void* workspace, size_t workspace_bytes, void* stream);
+                       const void* workspace, size_t workspace_bytes,
+                       const int32_t* doc_start, void* stream);
 int mmsp_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dout,
                      int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d,
                      float scale, int32_t causal, void* dq, float* dq_acc_opt,
-                     const void* workspace, size_t workspace_bytes, void* stream);
+                     const void* workspace, size_t workspace_bytes,
+                     const int32_t* doc_start, void* stream);
 
 /* Scratch bytes mmsp_attn_bwd needs for these sizes (0 on invalid sizes). */
 size_t mmsp_bwd_workspace_bytes(int64_t N, int32_t P, int32_t Hq, int32_t d);
@@ -240,7 +274,7 @@ int mmsp_attn_bwd_noalloc(const void* q, const void* k, const void* v,
                           int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d,
                           float scale, int32_t causal,
                           void* dq, void* dk, void* dv, float* dq_acc_opt,
-                          void* stream);
+                          const int32_t* doc_start, void* stream);
 
 /* Message of the calling thread's last failed call ("" if none). */
 const char* mmsp_last_error(void);

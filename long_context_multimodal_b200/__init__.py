@@ -22,6 +22,7 @@ from ._binding import (  # noqa: F401
     mmsp_attn_fwd,
     mmsp_bwd_workspace_bytes,
     mmsp_device_status,
+    mmsp_doc_starts,
     mmsp_last_error,
     mmsp_lse_merge,
     mmsp_selftest_bounded_wait,

@@ -41,22 +41,24 @@ _SIGS = {
     "mmsp_shard": ([c_void_p, c_void_p, c_int32, c_int64, c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
                     c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_void_p], c_int32),
     "mmsp_attn_fwd": ([c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32, c_int32, c_int32, c_float,
-                       c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_uint32, c_void_p], c_int32),
+                       c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_uint32, c_void_p, c_void_p],
+                      c_int32),
+    "mmsp_doc_starts": ([c_void_p, c_int32, c_int64, c_void_p, c_void_p], c_int32),
     "mmsp_lse_merge": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32,
                         c_void_p], c_int32),
     "mmsp_attn_bwd": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32,
                        c_int32, c_int32, c_float, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
-                       c_size_t, c_void_p], c_int32),
+                       c_size_t, c_void_p, c_void_p], c_int32),
     "mmsp_attn_bwd_prepare": ([c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32, c_int32, c_void_p, c_size_t,
                                c_void_p], c_int32),
     "mmsp_attn_bwd_dkdv": ([c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32, c_int32, c_int32,
-                            c_float, c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p], c_int32),
+                            c_float, c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p], c_int32),
     "mmsp_attn_bwd_dq": ([c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32, c_int32, c_int32,
-                          c_float, c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p], c_int32),
+                          c_float, c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p], c_int32),
     "mmsp_bwd_workspace_bytes": ([c_int64, c_int32, c_int32, c_int32], c_size_t),
     "mmsp_attn_bwd_noalloc": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32,
                                c_int32, c_int32, c_int32, c_float, c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
-                               c_void_p], c_int32),
+                               c_void_p, c_void_p], c_int32),
     "mmsp_last_error": ([], ctypes.c_char_p),
     "mmsp_device_status": ([c_void_p], c_int32),
     "mmsp_selftest_bounded_wait": ([c_int64, c_void_p], c_int32),
@@ -129,11 +131,18 @@ def mmsp_shard(seg_len, seg_kind, N, P, local2global=None, global2local=None, mo
 
 
 def mmsp_attn_fwd(q, k, v, N, P, Hq, Hkv, d, scale, causal, step_begin, step_end, o_acc, lse, o_out,
-                  flags, stream=None):
+                  flags, doc_start=None, stream=None):
     rc = _lib.mmsp_attn_fwd(_ptr(q), _ptr(k), _ptr(v), int(N), int(P), int(Hq), int(Hkv), int(d), float(scale),
                             int(causal), int(step_begin), int(step_end), _ptr(o_acc), _ptr(lse), _ptr(o_out),
-                            int(flags), _stream(stream))
+                            int(flags), _ptr(doc_start), _stream(stream))
     return _check("mmsp_attn_fwd", rc)
+
+
+def mmsp_doc_starts(doc_len, N, doc_start, stream=None):
+    """doc_start[g] (device int32 [N]) from host document lengths."""
+    dl = np.ascontiguousarray(np.asarray(doc_len, dtype=np.int32))
+    rc = _lib.mmsp_doc_starts(dl.ctypes.data_as(c_void_p), int(dl.size), int(N), _ptr(doc_start), _stream(stream))
+    return _check("mmsp_doc_starts", rc)
 
 
 def mmsp_lse_merge(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, H, d, stream=None):
@@ -143,10 +152,11 @@ def mmsp_lse_merge(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, H, d, stream=No
 
 
 def mmsp_attn_bwd(q, k, v, o, dout, lse, N, P, Hq, Hkv, d, scale, causal, dq, dk, dv, dq_acc_opt,
-                  workspace, workspace_bytes, stream=None):
+                  workspace, workspace_bytes, doc_start=None, stream=None):
     rc = _lib.mmsp_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), int(N), int(P), int(Hq),
                             int(Hkv), int(d), float(scale), int(causal), _ptr(dq), _ptr(dk), _ptr(dv),
-                            _ptr(dq_acc_opt), _ptr(workspace), int(workspace_bytes), _stream(stream))
+                            _ptr(dq_acc_opt), _ptr(workspace), int(workspace_bytes), _ptr(doc_start),
+                            _stream(stream))
     return _check("mmsp_attn_bwd", rc)
 
 
@@ -157,28 +167,28 @@ def mmsp_attn_bwd_prepare(o, dout, lse, N, P, Hq, d, workspace, workspace_bytes,
 
 
 def mmsp_attn_bwd_dkdv(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, dk, dv, workspace, workspace_bytes,
-                       stream=None):
+                       doc_start=None, stream=None):
     rc = _lib.mmsp_attn_bwd_dkdv(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), int(N), int(P), int(Hq), int(Hkv), int(d),
                                  float(scale), int(causal), _ptr(dk), _ptr(dv), _ptr(workspace),
-                                 int(workspace_bytes), _stream(stream))
+                                 int(workspace_bytes), _ptr(doc_start), _stream(stream))
     return _check("mmsp_attn_bwd_dkdv", rc)
 
 
 def mmsp_attn_bwd_dq(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, dq, dq_acc_opt, workspace, workspace_bytes,
-                     stream=None):
+                     doc_start=None, stream=None):
     rc = _lib.mmsp_attn_bwd_dq(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), int(N), int(P), int(Hq), int(Hkv), int(d),
                                float(scale), int(causal), _ptr(dq), _ptr(dq_acc_opt), _ptr(workspace),
-                               int(workspace_bytes), _stream(stream))
+                               int(workspace_bytes), _ptr(doc_start), _stream(stream))
     return _check("mmsp_attn_bwd_dq", rc)
 
 
 def mmsp_attn_bwd_noalloc(q, k, v, o, dout, lse, N, P, Hq, Hkv, d, scale, causal, dq, dk, dv, dq_acc_opt,
-                          stream=None):
+                          doc_start=None, stream=None):
     """Backward with the library's own fixed scratch (no allocation anywhere;
     see include/mmsp.h for the capacity and the sharing rules)."""
     rc = _lib.mmsp_attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), int(N), int(P),
                                     int(Hq), int(Hkv), int(d), float(scale), int(causal), _ptr(dq), _ptr(dk),
-                                    _ptr(dv), _ptr(dq_acc_opt), _stream(stream))
+                                    _ptr(dv), _ptr(dq_acc_opt), _ptr(doc_start), _stream(stream))
     return _check("mmsp_attn_bwd_noalloc", rc)
 
 

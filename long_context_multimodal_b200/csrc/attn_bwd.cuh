@@ -62,6 +62,7 @@ struct Params {
   float* dq_acc;        // [N][Hq][d] fp32 dQ or nullptr
   __nv_bfloat16* dk;    // [N][Hkv][d]
   __nv_bfloat16* dv;    // [N][Hkv][d]
+  const int32_t* doc_start;  // [N] global order, first position of each token's document; or null
   long long wait_cap;
 };
 
@@ -109,15 +110,20 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int64_t idx) {
   return u;
 }
 
-// Enumerates the (query tile, head) visits of a unit in ring order.
+// Enumerates the (query tile, head) visits of a unit in ring order. DOC:
+// queries carry document bounds (packed sequences); compiled out otherwise.
+template <bool DOC>
 struct VisitIter {
   int k, P, gk, causal, G, kvh, s, qc, t, tmax, hg, ntiles;
-  int64_t C, key0, qrow_base;
+  int64_t C, key0, qrow_base, kg0, kg1, qchunk0;
+  const int32_t* doc_start;
   bool in_chunk;
   int h, r, qcur;  // query head, rank, query chunk (0/1)
   int64_t q0;      // first query row of the tile within its chunk
   int64_t lrow0;   // first rank-local row of the tile
+  int64_t qglob0;  // global position of the tile's first query
   bool diag;
+  bool dmask;      // some query of the tile starts its document after a key of the unit
 
   __device__ __forceinline__ VisitIter(const Params& p, const Unit& u) {
     k = u.k;
@@ -136,6 +142,20 @@ struct VisitIter {
     key0 = u.key0;
     in_chunk = false;
     diag = false;
+    dmask = false;
+    doc_start = p.doc_start;
+    kg0 = (int64_t)u.gk * p.C + u.key0;
+    kg1 = (int64_t)u.gk * p.C + (u.key0 + BM - 1 < p.C - 1 ? u.key0 + BM - 1 : p.C - 1);
+  }
+
+  // Document test of the current query tile: false if every query's
+  // document starts after the unit's last key (nothing visible).
+  __device__ __forceinline__ bool doc_ok() {
+    if constexpr (!DOC) return true;
+    const int64_t qlast = qchunk0 + (q0 + BN - 1 < C - 1 ? q0 + BN - 1 : C - 1);
+    if (doc_start[qglob0] > kg1) return false;
+    dmask = doc_start[qlast] > kg0;
+    return true;
   }
 
   __device__ __forceinline__ bool next() {
@@ -148,11 +168,14 @@ struct VisitIter {
         }
         hg = 0;
         ++t;
-        if (t <= tmax) {
+        while (t <= tmax) {
           q0 = (int64_t)t * BN;
           lrow0 = qrow_base + q0;
-          continue;
+          qglob0 = qchunk0 + q0;
+          if (doc_ok()) break;
+          ++t;
         }
+        if (t <= tmax) continue;
         in_chunk = false;
       }
       if (s >= P) return false;
@@ -170,9 +193,15 @@ struct VisitIter {
       tmax = ntiles - 1;
       hg = 0;
       qrow_base = (int64_t)r * 2 * C + (int64_t)qcur * C;
-      q0 = (int64_t)t * BN;
-      lrow0 = qrow_base + q0;
-      in_chunk = true;
+      qchunk0 = (int64_t)gq * C;
+      while (t <= tmax) {
+        q0 = (int64_t)t * BN;
+        lrow0 = qrow_base + q0;
+        qglob0 = qchunk0 + q0;
+        if (doc_ok()) break;
+        ++t;
+      }
+      in_chunk = t <= tmax;
     }
   }
 };
@@ -193,6 +222,7 @@ struct SmemKV {
   static constexpr int ALLOC = BYTES;
 };
 
+template <bool DOC>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -277,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d_w(leader, sV + hf * HALF, &tmV, kv_full, hf * 64, u.kvh, krow);
       }
       ++ucnt;
-      VisitIter it(p, u);
+      VisitIter<DOC> it(p, u);
       while (it.next()) {
         const int st = vis & 1;
         const uint32_t use = vis >> 1;
@@ -336,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(kv_full, ucnt & 1, abort_flag, cap);
       ++ucnt;
       tc_fence_after();
-      VisitIter it(p, u);
+      VisitIter<DOC> it(p, u);
       bool has = it.next();
       bool first = true;
       if (has) {
@@ -394,17 +424,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit u = decode_unit(p, idx);
       const int64_t kin = u.key0 + row;  // key index within its chunk
       const bool key_ok = kin < p.C;
-      VisitIter it(p, u);
+      VisitIter<DOC> it(p, u);
       while (it.next()) {
         const int st = vis & 1;
         const float* lse2 = vec_g + st * 256;
         const float* dvec = lse2 + 128;
         // visible query columns: c >= cmin (diagonal); none for keys past C
-        int cmin = 0;
+        int cmin = 0, cmax = 128;  // visible query columns [cmin, cmax)
         if (!key_ok) cmin = 128;
         else if (it.diag) {
           const int64_t dmin = kin - it.q0;
           cmin = dmin <= 0 ? 0 : (dmin >= 128 ? 128 : (int)dmin);
+        }
+        if (DOC && it.dmask && key_ok) {
+          // first column whose document starts after this key (document
+          // starts are non-decreasing along the queries): binary search
+          const int64_t gkey = it.kg0 + row;
+          int lo = 0, hi = (int)(p.C - it.q0 < 128 ? p.C - it.q0 : 128);
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if ((int64_t)p.doc_start[it.qglob0 + mid] > gkey) hi = mid;
+            else lo = mid + 1;
+          }
+          cmax = lo;
         }
         mbar_wait(q_full(st), (vis >> 1) & 1, abort_flag, cap);  // LSE2/D arrive with Q
         // S^T -> P^T, written back as bf16 pairs over read columns
@@ -425,10 +467,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             float e1 = ex2_approx(fmaf(__uint_as_float(sr[j + 1]), sl2, -lv.y));
             float e2 = ex2_approx(fmaf(__uint_as_float(sr[j + 2]), sl2, -lv.z));
             float e3 = ex2_approx(fmaf(__uint_as_float(sr[j + 3]), sl2, -lv.w));
-            if (c < cmin) e0 = 0.f;
-            if (c + 1 < cmin) e1 = 0.f;
-            if (c + 2 < cmin) e2 = 0.f;
-            if (c + 3 < cmin) e3 = 0.f;
+            if (c < cmin || c >= cmax) e0 = 0.f;
+            if (c + 1 < cmin || c + 1 >= cmax) e1 = 0.f;
+            if (c + 2 < cmin || c + 2 >= cmax) e2 = 0.f;
+            if (c + 3 < cmin || c + 3 >= cmax) e3 = 0.f;
             pk[j / 2] = pack_bf16x2(e0, e1);
             pk[j / 2 + 1] = pack_bf16x2(e2, e3);
           }
@@ -548,11 +590,12 @@ __device__ __forceinline__ QItem decode_qitem(const Params& p, int64_t idx) {
 
 // K/V tiles a query tile visits, in ring order (rank r holds rank (r-s)
 // mod P's block at step s).
+template <bool DOC>
 struct KVIter {
   int r, P, gq, causal, s, ck, t, tmax, ntiles;
-  int64_t C, q0, base_row;
+  int64_t C, q0, base_row, kchunk0, lo_min, lo_max;
   bool in_chunk, diag;
-  int64_t kv_row;
+  int64_t kv_row, kglob0;
   int key0;
   bool mask;
 
@@ -570,6 +613,12 @@ struct KVIter {
     q0 = it.q0;
     in_chunk = false;
     diag = false;
+    lo_min = lo_max = 0;
+    if constexpr (DOC) {
+      const int64_t g0 = (int64_t)gq * C;
+      lo_min = p.doc_start[g0 + q0];
+      lo_max = p.doc_start[g0 + (q0 + BM - 1 < C - 1 ? q0 + BM - 1 : C - 1)];
+    }
   }
 
   __device__ __forceinline__ bool next() {
@@ -582,11 +631,13 @@ struct KVIter {
         const bool skip = causal && gk > gq;
         diag = causal && gk == gq;
         base_row = (int64_t)k * 2 * C + (int64_t)ck * C;
+        kchunk0 = (int64_t)gk * C;
         if (++ck == 2) {
           ck = 0;
           ++s;
         }
         if (skip) continue;
+        if (DOC && kchunk0 + C - 1 < lo_min) continue;  // whole chunk before every document
         int64_t last = q0 + BM - 1;
         if (last > C - 1) last = C - 1;
         tmax = diag ? (int)(last / BN) : ntiles - 1;
@@ -599,7 +650,10 @@ struct KVIter {
       }
       key0 = t * BN;
       ++t;
-      mask = (diag && (int64_t)key0 + BN - 1 > q0) || ((int64_t)key0 + BN > C);
+      kglob0 = kchunk0 + key0;
+      const int64_t klast = kchunk0 + ((int64_t)key0 + BN - 1 < C - 1 ? (int64_t)key0 + BN - 1 : C - 1);
+      if (DOC && klast < lo_min) continue;
+      mask = (diag && (int64_t)key0 + BN - 1 > q0) || ((int64_t)key0 + BN > C) || (DOC && kglob0 < lo_max);
       kv_row = base_row + key0;
       return true;
     }
@@ -619,6 +673,7 @@ struct SmemQ {
   static constexpr int ALLOC = BYTES;  // needs a 1024-aligned base (see SmemKV)
 };
 
+template <bool DOC>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -700,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d_w(leader, sDO + hf * HALF, &tmDO, q_full, hf * 64, it.h, (int)it.lrow0);
       }
       ++icnt;
-      KVIter ki(p, it);
+      KVIter<DOC> ki(p, it);
       while (ki.next()) {
         const int st = (int)(kc % NK);
         mbar_wait(k_empty(st), ((kc / NK) & 1) ^ 1, abort_flag, cap);
@@ -765,7 +820,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(q_full, icnt & 1, abort_flag, cap);
       ++icnt;
       tc_fence_after();
-      KVIter ki(p, it);
+      KVIter<DOC> ki(p, it);
       bool has = ki.next();
       uint32_t kcur = kc;
       if (has) {
@@ -824,11 +879,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t vrow = (((int64_t)it.h * p.P + it.r) * 2 + it.c) * p.Cp + qin;
       const float lse2 = p.lse2t[vrow];
       const float dval = p.dt[vrow];
-      KVIter ki(p, it);
+      const int64_t gq_row = (int64_t)(it.c ? 2 * p.P - 1 - it.r : it.r) * p.C + qin;
+      const int64_t lo_row = (DOC && qin < p.C) ? (int64_t)p.doc_start[gq_row] : 0;
+      KVIter<DOC> ki(p, it);
       bool any = false;
       while (ki.next()) {
         any = true;
-        int lim = 128;  // visible key columns of this row in the tile
+        int lim = 128, lb = 0;  // visible key columns of this row in the tile: [lb, lim)
         if (ki.mask) {
           int64_t l = p.C - ki.key0;
           if (ki.diag) {
@@ -836,6 +893,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             l = dl < l ? dl : l;
           }
           lim = l < 0 ? 0 : (l > 128 ? 128 : (int)l);
+          if (DOC) {
+            const int64_t b = lo_row - ki.kglob0;
+            lb = b < 0 ? 0 : (b > 128 ? 128 : (int)b);
+          }
         }
         const int b = scnt & 1;
         mbar_wait(s_full(b), (scnt >> 1) & 1, abort_flag, cap);
@@ -852,8 +913,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int c = (int)cq + 32 * h + j;
             float e0 = ex2_approx(fmaf(__uint_as_float(sr[j]), sl2, -lse2));
             float e1 = ex2_approx(fmaf(__uint_as_float(sr[j + 1]), sl2, -lse2));
-            if (c >= lim) e0 = 0.f;
-            if (c + 1 >= lim) e1 = 0.f;
+            if (c >= lim || c < lb) e0 = 0.f;
+            if (c + 1 >= lim || c + 1 < lb) e1 = 0.f;
             pk[16 * h + j / 2] = pack_bf16x2(e0, e1);
           }
         }

@@ -62,6 +62,7 @@ struct Params {
   float* o_acc;
   float* lse;
   __nv_bfloat16* o_out;
+  const int32_t* doc_start;  // [N] global order, first position of each token's document; or null
   long long wait_cap;
 };
 
@@ -96,13 +97,20 @@ __device__ __forceinline__ Item decode_item(const Params& p, int64_t idx) {
   return it;
 }
 
-// Enumerates the K/V tiles an item visits, in ring order.
+// Enumerates the K/V tiles an item visits, in ring order. DOC: rows carry
+// document bounds (packed sequences); compiled out otherwise.
+template <bool DOC>
 struct TileIter {
   int r, P, gq, causal, s, se, ck, t, tmax, ntiles;
   int64_t C, rowA0, base_row;
+  int32_t kchunk0;  // global position of the current K/V chunk (N < 2^31)
   bool validA, validB, in_chunk, diag;
+  // document bounds (global positions): the smallest and largest first key
+  // position over the rows of tiles A and B (0 without documents)
+  int32_t loA_min, loA_max, loB_min, loB_max;
   // current tile
   int64_t kv_row;
+  int32_t kglob0;
   int key0;
   bool actA, actB, maskA, maskB;
 
@@ -123,6 +131,18 @@ struct TileIter {
     validB = it.validB;
     in_chunk = false;
     diag = false;
+    loA_min = loA_max = loB_min = loB_max = 0;
+    if constexpr (DOC) {
+      const int32_t g0 = gq * (int32_t)C;
+      const int32_t a1 = (int32_t)(rowA0 + 127 < C - 1 ? rowA0 + 127 : C - 1);
+      loA_min = p.doc_start[g0 + (int32_t)rowA0];
+      loA_max = p.doc_start[g0 + a1];
+      if (validB) {
+        const int32_t b1 = (int32_t)(rowA0 + 255 < C - 1 ? rowA0 + 255 : C - 1);
+        loB_min = p.doc_start[g0 + (int32_t)rowA0 + 128];
+        loB_max = p.doc_start[g0 + b1];
+      }
+    }
   }
 
   __device__ __forceinline__ bool next() {
@@ -135,11 +155,15 @@ struct TileIter {
         const bool skip = causal && gk > gq;
         diag = causal && gk == gq;
         base_row = (int64_t)k * 2 * C + (int64_t)ck * C;
+        kchunk0 = gk * (int32_t)C;
         if (++ck == 2) {
           ck = 0;
           ++s;
         }
         if (skip) continue;
+        // whole chunk before every row's document
+        const int32_t klast_chunk = kchunk0 + (int32_t)C - 1;
+        if (DOC && klast_chunk < loA_min && (!validB || klast_chunk < loB_min)) continue;
         int64_t last = rowA0 + (validB ? 255 : 127);
         if (last > C - 1) last = C - 1;
         tmax = diag ? (int)(last / BN) : ntiles - 1;
@@ -152,12 +176,14 @@ struct TileIter {
       }
       key0 = t * BN;
       ++t;
-      actA = validA && (!diag || key0 <= rowA0 + 127);
-      actB = validB && (!diag || key0 <= rowA0 + 255);
+      kglob0 = kchunk0 + key0;
+      const int32_t klast = kchunk0 + (int32_t)((int64_t)key0 + BN - 1 < C - 1 ? (int64_t)key0 + BN - 1 : C - 1);
+      actA = validA && (!diag || key0 <= rowA0 + 127) && (!DOC || klast >= loA_min);
+      actB = validB && (!diag || key0 <= rowA0 + 255) && (!DOC || klast >= loB_min);
       if (!(actA || actB)) continue;
       const bool tail = (int64_t)key0 + BN > C;
-      maskA = (diag && (int64_t)key0 + BN - 1 > rowA0) || tail;
-      maskB = (diag && (int64_t)key0 + BN - 1 > rowA0 + 128) || tail;
+      maskA = (diag && (int64_t)key0 + BN - 1 > rowA0) || tail || (DOC && kglob0 < loA_max);
+      maskB = (diag && (int64_t)key0 + BN - 1 > rowA0 + 128) || tail || (DOC && kglob0 < loB_max);
       kv_row = base_row + key0;
       return true;
     }
@@ -176,7 +202,7 @@ struct Smem {
   static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
 };
 
-template <int D>
+template <int D, bool DOC>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Params p) {
@@ -255,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (it.validB) tma_load_3d_w(leader, sQ1 + hf * HALF, &tmQ, q_full, hf * 64, it.h, rowA + 128);
         }
         ++qcnt;
-        TileIter ti(p, it);
+        TileIter<DOC> ti(p, it);
         while (ti.next()) {
 #pragma unroll
           for (int kv = 0; kv < 2; ++kv) {
@@ -340,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++qcnt;
         tc_fence_after();
         first_pv[0] = first_pv[1] = true;
-        TileIter ti(p, it);
+        TileIter<DOC> ti(p, it);
         bool has = ti.next();
         if (has) {
           const int64_t kpos = pos++;
@@ -390,22 +416,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = grp ? it.validB : it.validA;
       if (!valid) continue;
       const int64_t rin = it.rowA0 + grp * 128 + row;  // row within the chunk
+      // first visible key (global position) of this row's document
+      const int32_t gqrow = (it.c ? 2 * p.P - 1 - it.r : it.r) * (int32_t)p.C + (int32_t)rin;
+      const int32_t lo_row = (DOC && rin < p.C) ? p.doc_start[gqrow] : 0;
       float m = -CUDART_INF_F, l = 0.f;
       int n_pv = 0;
-      TileIter ti(p, it);
+      TileIter<DOC> ti(p, it);
       while (ti.next()) {
         if (!(grp ? ti.actB : ti.actA)) continue;
         const bool msk = grp ? ti.maskB : ti.maskA;
         mbar_wait(s_full(grp), s_cnt & 1, abort_flag, cap);
         ++s_cnt;
         tc_fence_after();
-        int64_t lim = 128;  // visible columns of this row in the tile
+        int64_t lim = 128;  // visible columns of this row in the tile: [lb, lim)
+        int32_t lb = 0;
         if (msk) {
           lim = ti.C - ti.key0;
           if (ti.diag) {
             const int64_t dl = rin - ti.key0 + 1;
             lim = dl < lim ? dl : lim;
           }
+          if (DOC) lb = lo_row - ti.kglob0;
         }
         // pass 1: row max over the tile, 64 columns per TMEM round trip
         // The per-tile softmax, compiled twice: with the causal / ragged-tail
@@ -426,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 64; ++j) {
-              const float x = (!MK || 64 * h + j < lim) ? __uint_as_float(sr[j]) : -CUDART_INF_F;
+              const float x = (!MK || (64 * h + j < lim && 64 * h + j >= lb)) ? __uint_as_float(sr[j]) : -CUDART_INF_F;
               mxv[j & 7] = fmaxf(mxv[j & 7], x);
             }
           }
@@ -467,8 +498,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int j0 = 32 * q2 + 2 * u;
                 float e0 = ex2_approx(fmaf(__uint_as_float(sr[j0]), sl2, -mu));
                 float e1 = ex2_approx(fmaf(__uint_as_float(sr[j0 + 1]), sl2, -mu));
-                if (MK && 64 * h + j0 >= lim) e0 = 0.f;
-                if (MK && 64 * h + j0 + 1 >= lim) e1 = 0.f;
+                if (MK && (64 * h + j0 >= lim || 64 * h + j0 < lb)) e0 = 0.f;
+                if (MK && (64 * h + j0 + 1 >= lim || 64 * h + j0 + 1 < lb)) e1 = 0.f;
                 rsv[(2 * u) & 7] += e0;
                 rsv[(2 * u + 1) & 7] += e1;
                 pk[u] = pack_bf16x2_alu(e0, e1);

@@ -51,7 +51,7 @@ constexpr int kMaxDevices = 64;
 
 struct DeviceInfo {
   int sms = 0;
-  bool fwd_attr[2] = {false, false};
+  bool fwd_attr[4] = {false, false, false, false};
   bool bwd_attr[2] = {false, false};
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -199,6 +199,36 @@ int mmsp_shard(const int32_t* seg_len, const uint8_t* seg_kind, int32_t n_seg, i
   return ok();
 }
 
+int mmsp_doc_starts(const int32_t* doc_len, int32_t n_doc, int64_t N, int32_t* doc_start, void* stream) {
+  if (N < 0 || N > INT32_MAX) return fail(MMSP_EINVAL, "N must be in [0, 2^31-1]");
+  if (!doc_len || !doc_start) return fail(MMSP_EINVAL, "doc_len and doc_start must be non-NULL");
+  if ((uintptr_t)doc_start & 3u) return fail(MMSP_EINVAL, "doc_start must be 4-byte aligned");
+  if (N == 0) return ok();
+  if (n_doc < 1 || n_doc > MMSP_MAX_SEGMENTS)
+    return fail(MMSP_EINVAL, "n_doc must be in [1, %d] (got %d)", MMSP_MAX_SEGMENTS, n_doc);
+  static SegTable tab;
+  static std::mutex tab_mu;
+  std::lock_guard<std::mutex> lk(tab_mu);
+  int64_t acc = 0;
+  tab.n = n_doc;
+  for (int i = 0; i < n_doc; ++i) {
+    if (doc_len[i] < 1) return fail(MMSP_EINVAL, "document %d has length %d < 1", i, doc_len[i]);
+    tab.start[i] = (int32_t)acc;
+    tab.kind[i] = 0;
+    acc += doc_len[i];
+    if (acc > N) break;
+  }
+  if (acc != N) return fail(MMSP_EINVAL, "document lengths sum to %lld, expected N=%lld", (long long)acc, (long long)N);
+  tab.start[n_doc] = (int32_t)N;
+  int dev, sms, rc;
+  if ((rc = current_device(&dev)) || (rc = device_sms(dev, &sms))) return rc;
+  int64_t blocks = (N + 255) / 256;
+  if (blocks > 8LL * sms) blocks = 8LL * sms;
+  doc_starts_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(tab, (int32_t)N, doc_start);
+  MMSP_CUDA(cudaGetLastError());
+  return ok();
+}
+
 int mmsp_lse_merge(const float* o_a, const float* lse_a, const float* o_b, const float* lse_b, float* o_out,
                    float* lse_out, int64_t rows, int32_t H, int32_t d, void* stream) {
   if (rows < 0 || H < 1) return fail(MMSP_EINVAL, "rows must be >= 0 and H >= 1");
@@ -225,12 +255,37 @@ int mmsp_lse_merge(const float* o_a, const float* lse_a, const float* o_b, const
   return ok();
 }
 
+}  // extern "C"
+
+namespace {
+// One forward variant: shared-memory opt-in once per device, then launch.
+template <int D, bool DOC>
+int launch_fwd(int dev, int vi, int64_t grid, cudaStream_t st, const CUtensorMap& tq, const CUtensorMap& tk,
+               const CUtensorMap& tv, const fwd::Params& p) {
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_dev[dev].fwd_attr[vi]) {
+      MMSP_CUDA(cudaFuncSetAttribute(fwd::attn_fwd_kernel<D, DOC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     fwd::Smem<D>::ALLOC));
+      g_dev[dev].fwd_attr[vi] = true;
+    }
+  }
+  fwd::attn_fwd_kernel<D, DOC><<<(unsigned)grid, fwd::kThreads, fwd::Smem<D>::ALLOC, st>>>(tq, tk, tv, p);
+  MMSP_CUDA(cudaGetLastError());
+  return MMSP_OK;
+}
+}  // namespace
+
+extern "C" {
+
 int mmsp_attn_fwd(const void* q, const void* k, const void* v, int64_t N, int32_t P, int32_t Hq, int32_t Hkv,
                   int32_t d, float scale, int32_t causal, int32_t step_begin, int32_t step_end, float* o_acc,
-                  float* lse, void* o_out, uint32_t flags, void* stream) {
+                  float* lse, void* o_out, uint32_t flags, const int32_t* doc_start, void* stream) {
   int rc = check_common(N, P);
   if (rc) return rc;
   if ((rc = check_heads(Hq, Hkv, d))) return rc;
+  if (doc_start && causal != 1) return fail(MMSP_EINVAL, "doc_start needs causal = 1");
+  if (doc_start && ((uintptr_t)doc_start & 3u)) return fail(MMSP_EINVAL, "doc_start must be 4-byte aligned");
   if (flags & ~(MMSP_ACCUMULATE | MMSP_FINALIZE)) return fail(MMSP_EINVAL, "unknown flags 0x%x", flags);
   if (!(scale > 0.f) || !std::isfinite(scale)) return fail(MMSP_EINVAL, "scale must be finite and > 0");
   if (causal != 0 && causal != 1) return fail(MMSP_EINVAL, "causal must be 0 or 1");
@@ -266,27 +321,18 @@ int mmsp_attn_fwd(const void* q, const void* k, const void* v, int64_t N, int32_
   p.o_acc = o_acc;
   p.lse = lse;
   p.o_out = static_cast<__nv_bfloat16*>(o_out);
+  p.doc_start = doc_start;
   p.wait_cap = kWaitCapCycles;
   const int64_t grid = p.n_items < sms ? p.n_items : sms;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int di = d == 128 ? 1 : 0;
-  {
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_dev[dev].fwd_attr[di]) {
-      if (d == 128)
-        MMSP_CUDA(cudaFuncSetAttribute(fwd::attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       fwd::Smem<128>::ALLOC));
-      else
-        MMSP_CUDA(cudaFuncSetAttribute(fwd::attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       fwd::Smem<64>::ALLOC));
-      g_dev[dev].fwd_attr[di] = true;
-    }
-  }
+  const int vi = (d == 128 ? 2 : 0) + (doc_start ? 1 : 0);
   if (d == 128)
-    fwd::attn_fwd_kernel<128><<<(unsigned)grid, fwd::kThreads, fwd::Smem<128>::ALLOC, st>>>(tq, tk, tv, p);
+    rc = doc_start ? launch_fwd<128, true>(dev, vi, grid, st, tq, tk, tv, p)
+                   : launch_fwd<128, false>(dev, vi, grid, st, tq, tk, tv, p);
   else
-    fwd::attn_fwd_kernel<64><<<(unsigned)grid, fwd::kThreads, fwd::Smem<64>::ALLOC, st>>>(tq, tk, tv, p);
-  MMSP_CUDA(cudaGetLastError());
+    rc = doc_start ? launch_fwd<64, true>(dev, vi, grid, st, tq, tk, tv, p)
+                   : launch_fwd<64, false>(dev, vi, grid, st, tq, tk, tv, p);
+  if (rc) return rc;
   return ok();
 }
 
@@ -357,13 +403,15 @@ extern "C" size_t mmsp_bwd_workspace_bytes(int64_t N, int32_t P, int32_t Hq, int
 namespace {
 // Shared checks of the backward stages (sizes, scale, workspace).
 int bwd_check(int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d, float scale, int32_t causal,
-              const void* workspace, size_t workspace_bytes) {
+              const void* workspace, size_t workspace_bytes, const int32_t* doc_start = nullptr) {
   int rc = check_common(N, P);
   if (rc) return rc;
   if ((rc = check_heads(Hq, Hkv, d))) return rc;
   if (d != 128) return fail(MMSP_EUNSUPPORTED, "the backward supports d = 128 (got %d)", d);
   if (!(scale > 0.f) || !std::isfinite(scale)) return fail(MMSP_EINVAL, "scale must be finite and > 0");
   if (causal != 0 && causal != 1) return fail(MMSP_EINVAL, "causal must be 0 or 1");
+  if (doc_start && causal != 1) return fail(MMSP_EINVAL, "doc_start needs causal = 1");
+  if (doc_start && ((uintptr_t)doc_start & 3u)) return fail(MMSP_EINVAL, "doc_start must be 4-byte aligned");
   if (N == 0) return MMSP_OK;
   const BwdLayout Lw = bwd_layout(N, P, Hq, d);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -408,9 +456,13 @@ int bwd_setup(const void* q, const void* k, const void* v, const void* dout, int
   p->wait_cap = kWaitCapCycles;
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_dev[dev].bwd_attr[1]) {
-    MMSP_CUDA(cudaFuncSetAttribute(bwd::attn_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    MMSP_CUDA(cudaFuncSetAttribute(bwd::attn_bwd_dkdv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    bwd::SmemKV::ALLOC));
-    MMSP_CUDA(cudaFuncSetAttribute(bwd::attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    MMSP_CUDA(cudaFuncSetAttribute(bwd::attn_bwd_dkdv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   bwd::SmemKV::ALLOC));
+    MMSP_CUDA(cudaFuncSetAttribute(bwd::attn_bwd_dq_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   bwd::SmemQ::ALLOC));
+    MMSP_CUDA(cudaFuncSetAttribute(bwd::attn_bwd_dq_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    bwd::SmemQ::ALLOC));
     g_dev[dev].bwd_attr[1] = true;
   }
@@ -441,8 +493,9 @@ extern "C" int mmsp_attn_bwd_prepare(const void* o, const void* dout, const floa
 
 extern "C" int mmsp_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout, int64_t N,
                                   int32_t P, int32_t Hq, int32_t Hkv, int32_t d, float scale, int32_t causal,
-                                  void* dk, void* dv, const void* workspace, size_t workspace_bytes, void* stream) {
-  int rc = bwd_check(N, P, Hq, Hkv, d, scale, causal, workspace, workspace_bytes);
+                                  void* dk, void* dv, const void* workspace, size_t workspace_bytes,
+                                  const int32_t* doc_start, void* stream) {
+  int rc = bwd_check(N, P, Hq, Hkv, d, scale, causal, workspace, workspace_bytes, doc_start);
   if (rc) return rc;
   if (!q || !k || !v || !dout || !dk || !dv) return fail(MMSP_EINVAL, "q, k, v, dout, dk, dv must be non-NULL");
   if (!all_aligned16({q, k, v, dout, dk, dv})) return fail(MMSP_EINVAL, "all tensors must be 16-byte aligned");
@@ -454,17 +507,23 @@ extern "C" int mmsp_attn_bwd_dkdv(const void* q, const void* k, const void* v, c
     return rc;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.doc_start = doc_start;
   const int64_t grid = p.n_units < sms ? p.n_units : sms;
-  bwd::attn_bwd_dkdv_kernel<<<(unsigned)grid, bwd::kThreads, bwd::SmemKV::ALLOC, static_cast<cudaStream_t>(stream)>>>(
-      tq, tk, tv, tdo, p);
+  if (doc_start)
+    bwd::attn_bwd_dkdv_kernel<true><<<(unsigned)grid, bwd::kThreads, bwd::SmemKV::ALLOC,
+                                      static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, tdo, p);
+  else
+    bwd::attn_bwd_dkdv_kernel<false><<<(unsigned)grid, bwd::kThreads, bwd::SmemKV::ALLOC,
+                                       static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, tdo, p);
   MMSP_CUDA(cudaGetLastError());
   return ok();
 }
 
 extern "C" int mmsp_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dout, int64_t N, int32_t P,
                                 int32_t Hq, int32_t Hkv, int32_t d, float scale, int32_t causal, void* dq,
-                                float* dq_acc_opt, const void* workspace, size_t workspace_bytes, void* stream) {
-  int rc = bwd_check(N, P, Hq, Hkv, d, scale, causal, workspace, workspace_bytes);
+                                float* dq_acc_opt, const void* workspace, size_t workspace_bytes,
+                                const int32_t* doc_start, void* stream) {
+  int rc = bwd_check(N, P, Hq, Hkv, d, scale, causal, workspace, workspace_bytes, doc_start);
   if (rc) return rc;
   if (!q || !k || !v || !dout || !dq) return fail(MMSP_EINVAL, "q, k, v, dout, dq must be non-NULL");
   if (!all_aligned16({q, k, v, dout, dq, dq_acc_opt})) return fail(MMSP_EINVAL, "all tensors must be 16-byte aligned");
@@ -476,9 +535,14 @@ extern "C" int mmsp_attn_bwd_dq(const void* q, const void* k, const void* v, con
     return rc;
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dq_acc = dq_acc_opt;
+  p.doc_start = doc_start;
   const int64_t grid = p.n_items < sms ? p.n_items : sms;
-  bwd::attn_bwd_dq_kernel<<<(unsigned)grid, bwd::kThreads, bwd::SmemQ::ALLOC, static_cast<cudaStream_t>(stream)>>>(
-      tq, tk, tv, tdo, p);
+  if (doc_start)
+    bwd::attn_bwd_dq_kernel<true><<<(unsigned)grid, bwd::kThreads, bwd::SmemQ::ALLOC,
+                                    static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, tdo, p);
+  else
+    bwd::attn_bwd_dq_kernel<false><<<(unsigned)grid, bwd::kThreads, bwd::SmemQ::ALLOC,
+                                     static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, tdo, p);
   MMSP_CUDA(cudaGetLastError());
   return ok();
 }
@@ -486,8 +550,8 @@ extern "C" int mmsp_attn_bwd_dq(const void* q, const void* k, const void* v, con
 extern "C" int mmsp_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                              const float* lse, int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d, float scale,
                              int32_t causal, void* dq, void* dk, void* dv, float* dq_acc_opt, void* workspace,
-                             size_t workspace_bytes, void* stream) {
-  int rc = bwd_check(N, P, Hq, Hkv, d, scale, causal, workspace, workspace_bytes);
+                             size_t workspace_bytes, const int32_t* doc_start, void* stream) {
+  int rc = bwd_check(N, P, Hq, Hkv, d, scale, causal, workspace, workspace_bytes, doc_start);
   if (rc) return rc;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv)
     return fail(MMSP_EINVAL, "q, k, v, o, dout, lse, dq, dk, dv must be non-NULL");
@@ -496,10 +560,10 @@ extern "C" int mmsp_attn_bwd(const void* q, const void* k, const void* v, const 
   if (N == 0) return ok();
   if ((rc = mmsp_attn_bwd_prepare(o, dout, lse, N, P, Hq, d, workspace, workspace_bytes, stream))) return rc;
   if ((rc = mmsp_attn_bwd_dkdv(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, dk, dv, workspace, workspace_bytes,
-                               stream)))
+                               doc_start, stream)))
     return rc;
   return mmsp_attn_bwd_dq(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, dq, dq_acc_opt, workspace, workspace_bytes,
-                          stream);
+                          doc_start, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -531,12 +595,12 @@ int scratch_address(int dev, void** out) {
 extern "C" int mmsp_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
                                      const float* lse, int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d,
                                      float scale, int32_t causal, void* dq, void* dk, void* dv, float* dq_acc_opt,
-                                     void* stream) {
+                                     const int32_t* doc_start, void* stream) {
   int rc = check_common(N, P);
   if (rc) return rc;
   if ((rc = check_heads(Hq, Hkv, d))) return rc;
   if (N == 0) return mmsp_attn_bwd(q, k, v, o, dout, lse, N, P, Hq, Hkv, d, scale, causal, dq, dk, dv, dq_acc_opt,
-                                   nullptr, 0, stream);
+                                   nullptr, 0, doc_start, stream);
   const size_t need = mmsp_bwd_workspace_bytes(N, P, Hq, d);
   if (need > (size_t)MMSP_NOALLOC_SCRATCH_BYTES)
     return fail(MMSP_EINVAL, "sizes need %zu bytes of scratch; mmsp_attn_bwd_noalloc holds at most %zu (use "
@@ -546,5 +610,5 @@ extern "C" int mmsp_attn_bwd_noalloc(const void* q, const void* k, const void* v
   void* scratch = nullptr;
   if ((rc = scratch_address(dev, &scratch))) return rc;
   return mmsp_attn_bwd(q, k, v, o, dout, lse, N, P, Hq, Hkv, d, scale, causal, dq, dk, dv, dq_acc_opt, scratch,
-                       (size_t)MMSP_NOALLOC_SCRATCH_BYTES, stream);
+                       (size_t)MMSP_NOALLOC_SCRATCH_BYTES, doc_start, stream);
 }

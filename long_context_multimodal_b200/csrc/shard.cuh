@@ -64,6 +64,17 @@ __global__ void __launch_bounds__(256) shard_maps_kernel(const __grid_constant__
   }
 }
 
+// doc_start[g] = first position of the document holding global position g
+// (the document table is the segment table of the packed sequence).
+__global__ void __launch_bounds__(256) doc_starts_kernel(const __grid_constant__ SegTable tab, int32_t N,
+                                                         int32_t* __restrict__ doc_start) {
+  __shared__ int32_t s_start[kMaxSegments + 1];
+  for (int i = threadIdx.x; i <= tab.n; i += blockDim.x) s_start[i] = tab.start[i];
+  __syncthreads();
+  for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < N; g += (int64_t)gridDim.x * blockDim.x)
+    doc_start[g] = s_start[seg_of(s_start, tab.n, (int32_t)g)];
+}
+
 // One block: visual-token prefix over segments, then per rank the text and
 // visual counts of its two chunks.
 __global__ void __launch_bounds__(256) shard_counts_kernel(const __grid_constant__ SegTable tab, int32_t N,

@@ -127,6 +127,32 @@ def random_segments(N: int, seed: int, max_len: int = 700) -> Tuple[np.ndarray, 
     return np.asarray(lens, np.int32), np.asarray(kinds, np.uint8)
 
 
+def packed_documents(N: int, seed: int, max_frames: int = 6, text_max: int = 300
+                     ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """A seeded packed buffer of N tokens made of several short videos, each
+    a document of (prompt text, f frames of FRAME_TOKENS visual tokens,
+    answer text); the last document is cut at N. Returns (doc_len, seg_len,
+    seg_kind): the document lengths and the matching segment table."""
+    rng = np.random.default_rng(seed)
+    docs, lens, kinds = [], [], []
+    left = N
+    while left > 0:
+        parts = [(int(rng.integers(1, text_max + 1)), TEXT)]
+        parts += [(FRAME_TOKENS, VISUAL)] * int(rng.integers(1, max_frames + 1))
+        parts.append((int(rng.integers(1, 65)), TEXT))
+        used = 0
+        for L, kind in parts:
+            L = min(L, left - used)
+            if L <= 0:
+                break
+            lens.append(L)
+            kinds.append(kind)
+            used += L
+        docs.append(used)
+        left -= used
+    return np.asarray(docs, np.int32), np.asarray(lens, np.int32), np.asarray(kinds, np.uint8)
+
+
 def make_tensors(N: int, hq: int, hkv: int, d: int, seed: int, visual_mask,
                  device="cpu", with_dout: bool = False):
     """Q, K, V (and dO) as bf16 torch tensors [N, H, d], drawn in that order.

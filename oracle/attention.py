@@ -51,6 +51,22 @@ def _f64(x):
     return np.asarray(x, dtype=np.float64)
 
 
+def document_starts(doc_len):
+    """doc_start[g] for a packed sequence given as document lengths: the
+    position where the document holding g begins ("LongVILA Guide",
+    section "Critical Operational Best Practices", dynamic sequence packing:
+    several videos share one buffer and the attention mask resets between
+    them). Written as a plain loop over documents."""
+    out = []
+    pos = 0
+    for L in np.asarray(doc_len, np.int64).tolist():
+        if L < 1:
+            raise ValueError("document lengths must be >= 1")
+        out.extend([pos] * L)
+        pos += L
+    return np.asarray(out, np.int64)
+
+
 def _visible(jmax, rows, lo):
     """[R, jmax] mask: key j visible to row i iff lo_i <= j <= i (lo_i = 0
     without documents)."""
@@ -192,9 +208,10 @@ def causal_attention_bwd(q, k, v, do, scale=None, block: int = 512, doc_start=No
     return {"O": O, "LSE": LSE, "D": Dm, "dQ": dQ, "dK": dK, "dV": dV}
 
 
-def attention_bwd_rows(q_rows, k, v, do_rows, rows, scale=None, block: int = 64):
+def attention_bwd_rows(q_rows, k, v, do_rows, rows, scale=None, block: int = 64, doc_start=None):
     """dQ (and O, LSE) for selected global rows: row i needs only keys <= i.
-    q_rows and do_rows [R,Hq,d] are the caller-gathered rows at `rows`."""
+    q_rows and do_rows [R,Hq,d] are the caller-gathered rows at `rows`;
+    doc_start as in causal_attention."""
     q_rows, do_rows = _f64(q_rows), _f64(do_rows)
     rows = np.asarray(rows, np.int64)
     R, hq, d = q_rows.shape
@@ -213,21 +230,22 @@ def attention_bwd_rows(q_rows, k, v, do_rows, rows, scale=None, block: int = 64)
                 continue
             for b0 in range(0, R, block):
                 sel = np.arange(b0, min(R, b0 + block))
-                o, lse, _, dq, _, _ = _rows_backward(q_rows[sel, h], do_rows[sel, h], rows[sel], K, V, scale)
+                lo = None if doc_start is None else np.asarray(doc_start)[rows[sel]]
+                o, lse, _, dq, _, _ = _rows_backward(q_rows[sel, h], do_rows[sel, h], rows[sel], K, V, scale, lo)
                 dQ[sel, h] = dq
                 O[sel, h] = o
                 LSE[sel, h] = lse
     return {"O": O, "LSE": LSE, "dQ": dQ}
 
 
-def attention_bwd_keys(q_tail, k, v, do_tail, keys, scale=None, block: int = 64):
+def attention_bwd_keys(q_tail, k, v, do_tail, keys, scale=None, block: int = 64, doc_start=None):
     """dK and dV for selected global key positions.
 
     Key j receives contributions from rows i >= j only. q_tail and do_tail
     hold the rows [j0, N) of Q and dO, where j0 = min(keys) and N = len(k);
     those rows are computed in full (their LSE and D over keys <= i) and
     their terms are summed into the requested keys. Cheap only when the keys
-    lie near the end.
+    lie near the end. doc_start as in causal_attention.
     """
     keys = np.asarray(keys, np.int64)
     N = k.shape[0]
@@ -249,7 +267,9 @@ def attention_bwd_keys(q_tail, k, v, do_tail, keys, scale=None, block: int = 64)
                 continue
             for i0 in range(j0, N, block):
                 rows = np.arange(i0, min(N, i0 + block))
-                _, _, _, _, p, ds = _rows_backward(q_tail[rows - j0, h], do_tail[rows - j0, h], rows, K, V, scale)
+                lo = None if doc_start is None else np.asarray(doc_start)[rows]
+                _, _, _, _, p, ds = _rows_backward(q_tail[rows - j0, h], do_tail[rows - j0, h], rows, K, V, scale,
+                                                   lo)
                 sel = np.nonzero(keys <= rows.max())[0]
                 dV[sel, kh] += p[:, keys[sel]].T @ do_tail[rows - j0, h]
                 dK[sel, kh] += scale * (ds[:, keys[sel]].T @ q_tail[rows - j0, h])

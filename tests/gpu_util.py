@@ -33,7 +33,7 @@ def shard_rows(x, N, P, inverse=False):
 
 
 def run_forward(q, k, v, P, causal=1, step_begin=0, step_end=None, flags=None, scale=None,
-                o_acc=None, lse=None):
+                o_acc=None, lse=None, doc_start=None):
     """q, k, v: rank-local CUDA bf16 [N, H, d]. Returns (o_acc fp32, lse, o_out bf16)."""
     m = lib()
     N, hq, d = q.shape
@@ -50,7 +50,7 @@ def run_forward(q, k, v, P, causal=1, step_begin=0, step_end=None, flags=None, s
         lse = torch.full((N, hq), float("nan"), device=q.device, dtype=torch.float32)
     o_out = torch.full((N, hq, d), float("nan"), device=q.device, dtype=torch.bfloat16)
     m.mmsp_attn_fwd(q, k, v, N, P, hq, hkv, d, scale, causal, step_begin, step_end, o_acc, lse,
-                    o_out if flags & m.MMSP_FINALIZE else None, flags)
+                    o_out if flags & m.MMSP_FINALIZE else None, flags, doc_start=doc_start)
     m.mmsp_device_status()
     return o_acc, lse, o_out
 
@@ -103,7 +103,7 @@ def compare_grad(g, g_ref, what):
     return float(mx), float(mn)
 
 
-def run_backward(ql, kl, vl, o_out, dol, lse, P, causal=1, fp32_dq=False):
+def run_backward(ql, kl, vl, o_out, dol, lse, P, causal=1, fp32_dq=False, doc_start=None):
     """Rank-local inputs; returns (dq bf16, dk bf16, dv bf16, dq fp32 or None)."""
     m = lib()
     N, hq, d = ql.shape
@@ -115,6 +115,6 @@ def run_backward(ql, kl, vl, o_out, dol, lse, P, causal=1, fp32_dq=False):
     dv = torch.full_like(vl, float("nan"))
     dq32 = torch.full((N, hq, d), float("nan"), device=ql.device) if fp32_dq else None
     m.mmsp_attn_bwd(ql, kl, vl, o_out, dol, lse, N, P, hq, hkv, d, 1.0 / math.sqrt(d), causal, dq, dk, dv, dq32,
-                    ws, ws_bytes)
+                    ws, ws_bytes, doc_start=doc_start)
     m.mmsp_device_status()
     return dq, dk, dv, dq32

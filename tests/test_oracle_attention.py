@@ -121,6 +121,18 @@ def _doc_start(lengths):
     return np.asarray(out, np.int64)
 
 
+def test_document_starts_by_hand():
+    """Worked by hand from the definition (first position of each token's
+    document)."""
+    np.testing.assert_array_equal(A.document_starts([3, 1, 2]), [0, 0, 0, 3, 4, 4])
+    np.testing.assert_array_equal(A.document_starts([1, 1, 1]), [0, 1, 2])
+    np.testing.assert_array_equal(A.document_starts([5]), [0] * 5)
+    assert A.document_starts([]).size == 0
+    with pytest.raises(ValueError):
+        A.document_starts([2, 0, 1])
+    np.testing.assert_array_equal(A.document_starts([7, 1, 30]), _doc_start([7, 1, 30]))
+
+
 def test_document_mask_equals_separate_documents():
     """Packed sequence with attention reset at document boundaries = plain
     causal attention of each document on its own (brute force)."""

@@ -98,3 +98,22 @@ def test_document_mask_backward_equals_separate_documents():
         for name in ("O", "dQ", "dK", "dV"):
             np.testing.assert_allclose(g[name][sl], gd[name], atol=1e-12)
         pos += L
+
+
+def test_document_sampled_helpers_agree_with_whole_backward():
+    """attention_bwd_rows / attention_bwd_keys with documents equal the
+    whole-sequence backward (itself pinned to per-document attention)."""
+    lengths = [30, 5, 1, 40, 24]
+    N = sum(lengths)
+    q, k, v, do = _inputs(N, 4, 2, 8, 23)
+    ds = A.document_starts(lengths)
+    g = A.causal_attention_bwd(q, k, v, do, block=16, doc_start=ds)
+    rows = np.array([0, 29, 30, 35, 36, 50, 99])
+    r = A.attention_bwd_rows(q[rows], k, v, do[rows], rows, block=3, doc_start=ds)
+    np.testing.assert_allclose(r["dQ"], g["dQ"][rows], atol=1e-12)
+    np.testing.assert_allclose(r["O"], g["O"][rows], atol=1e-12)
+    np.testing.assert_allclose(r["LSE"], g["LSE"][rows], atol=1e-12)
+    keys = np.array([70, 75, 76, 99])
+    kk = A.attention_bwd_keys(q[70:], k, v, do[70:], keys, block=9, doc_start=ds)
+    np.testing.assert_allclose(kk["dK"], g["dK"][keys], atol=1e-12)
+    np.testing.assert_allclose(kk["dV"], g["dV"][keys], atol=1e-12)
