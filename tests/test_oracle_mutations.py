@@ -31,3 +31,30 @@ def test_dropped_merge_weight_is_caught():
     assert not np.allclose(wrong, g["o_out"])
     o, _ = M.lse_merge(oa, g["lse_a"][0], ob, g["lse_b"][0])
     assert np.allclose(o, g["o_out"])
+
+
+def test_rope_wrong_frequency_exponent_is_caught(monkeypatch):
+    import test_oracle_rope as TR
+    from oracle import rope as R
+    monkeypatch.setattr(R, "inv_freq", lambda d, theta: np.array([theta ** (-1.0 * i / d) for i in range(d // 2)]))
+    with pytest.raises(AssertionError):
+        TR.test_hand_worked_values()
+
+
+def test_rope_wrong_rotation_sign_is_caught(monkeypatch):
+    import test_oracle_rope as TR
+    from oracle import rope as R
+    real = R.rope
+    monkeypatch.setattr(R, "rope", lambda x, pos, theta=1e7, interleaved=False, inverse=False:
+                        real(x, pos, theta, interleaved, not inverse))
+    with pytest.raises(AssertionError):
+        TR.test_complex_multiplication_form(False)
+
+
+def test_rope_swapped_pairing_is_caught(monkeypatch):
+    import test_oracle_rope as TR
+    from oracle import rope as R
+    real = R.pair_index
+    monkeypatch.setattr(R, "pair_index", lambda d, interleaved: real(d, not interleaved))
+    with pytest.raises(AssertionError):
+        TR.test_hand_worked_values()
