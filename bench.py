@@ -356,6 +356,24 @@ def run_gpu(args):
     e2e_ms = e0.elapsed_time(e1) / e_steps
     m.mmsp_device_status(stream)
 
+    # ---------------- the RoPE-fused shard gather of Q (theta = 1e7), timed
+    # on its own next to the plain gather it replaces (not part of the step:
+    # the configured workload gives Q and K directly)
+    def time_calls(fn, reps=5):
+        fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        b.synchronize()
+        return a.elapsed_time(b) / reps
+
+    rope_ms = time_calls(lambda: m.mmsp_shard_rope(path.q, path.ql, w.N, w.P, w.hq, w.d, 1e7, False, stream=stream))
+    plain_ms = time_calls(lambda: m.mmsp_shard(None, None, w.N, w.P, src=path.q, dst=path.ql,
+                                               row_bytes=w.hq * w.d * 2, stream=stream))
+    m.mmsp_device_status(stream)
+
     # ---------------- max over ranks
     ms_total, e2e_ms, fwd_ms, bwd_ms, dkdv_ms, dq_ms = max_over_ranks(
         [ms_total, e2e_ms, fwd_ms, bwd_ms, dkdv_ms, dq_ms], ws, dev)
@@ -370,6 +388,8 @@ def run_gpu(args):
         dkdv_flops = 2.0 * w.fwd_flops()
         achieved = dkdv_flops / (dkdv_ms * 1e-3) / 1e12
         traffic = profiled_traffic(f"attn_bwd_dkdv_{w.name}.md", ["attn_bwd.cuh", "ptx.cuh"])
+        hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        rope_bytes = 2.0 * w.N * w.hq * w.d * 2  # read + write of Q, bf16
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -389,6 +409,10 @@ def run_gpu(args):
                           "bwd_total": bwd_ms},
             "e2e": {"value": flops * ws / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
+            "rope_gather": {"kernel": "shard_rope_kernel<128, half pairs> on Q, theta = 1e7", "bound": "hbm",
+                            "achieved": rope_bytes / (rope_ms * 1e-3) / 1e9, "unit": "GB/s",
+                            "peak": hbm_peak, "frac": rope_bytes / (rope_ms * 1e-3) / 1e9 / hbm_peak,
+                            "bytes_per_launch": rope_bytes, "ms": rope_ms, "plain_gather_ms": plain_ms},
             "gpu_launches": path.launches_per_step * args.steps,
             "clocks": clocks,
             "outputs_finite": ok,

@@ -92,6 +92,35 @@ int mmsp_shard(const int32_t* seg_len, const uint8_t* seg_kind, int32_t n_seg,
                void* stream);
 
 /*
+ * mmsp_shard_rope -- the shard gather of Q or K rows with the rotary
+ * position embedding applied on the way (inverse == 0), or the transposed
+ * rotation applied while scattering gradient rows back (inverse != 0).
+ *
+ * Source: "LongVILA Guide" (aifetchly), three-stage curriculum, Stage 2
+ * (RoPE base theta raised from 10,000 to 10^7) and section "Distributed
+ * Training Configuration" (RoPE base 10,000,000). The pages print no
+ * formula; this is the standard rotary embedding: pair (a, b) of each head
+ * vector turned by phi_i = pos * theta^(-2i/d), i < d/2:
+ *   a' = a cos(phi_i) - b sin(phi_i),  b' = a sin(phi_i) + b cos(phi_i).
+ *
+ *   src, dst      DEVICE bf16 [N][H][d], 16-byte aligned, not overlapping.
+ *                 inverse == 0: dst[l] = R(pos(g)) src[g] with g =
+ *                 local2global(l) (global -> rank-local, as mmsp_shard);
+ *                 inverse != 0: dst[g] = R(pos(g))^T src[l] (rank-local ->
+ *                 global; the gradient of the forward gather).
+ *   N, P          as mmsp_shard. H >= 1 heads; d in {8,16,32,64,128,256}.
+ *   theta         base, finite and > 1 (10^7 for the long-context stage).
+ *   interleaved   0: pairs (i, i + d/2); 1: pairs (2i, 2i + 1).
+ *   doc_start     DEVICE int32 [N] (see mmsp_doc_starts) or NULL: pos(g) =
+ *                 g - doc_start[g] (positions restart per packed document)
+ *                 or g.
+ * fp64 angle and range reduction, fp32 rotation, bf16 (RNE) result.
+ */
+int mmsp_shard_rope(const void* src, void* dst, int64_t N, int32_t P,
+                    int32_t H, int32_t d, double theta, int32_t interleaved,
+                    const int32_t* doc_start, int32_t inverse, void* stream);
+
+/*
  * mmsp_attn_fwd -- blockwise causal attention of every virtual rank's queries
  * over the K/V blocks it holds at ring steps [step_begin, step_end), merged
  * across steps with the online-softmax (log-sum-exp) combine.

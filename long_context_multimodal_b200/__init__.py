@@ -27,6 +27,7 @@ from ._binding import (  # noqa: F401
     mmsp_lse_merge,
     mmsp_selftest_bounded_wait,
     mmsp_shard,
+    mmsp_shard_rope,
     mmsp_version,
     exported_symbols,
 )

@@ -44,6 +44,8 @@ _SIGS = {
                        c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_uint32, c_void_p, c_void_p],
                       c_int32),
     "mmsp_doc_starts": ([c_void_p, c_int32, c_int64, c_void_p, c_void_p], c_int32),
+    "mmsp_shard_rope": ([c_void_p, c_void_p, c_int64, c_int32, c_int32, c_int32, ctypes.c_double, c_int32, c_void_p,
+                         c_int32, c_void_p], c_int32),
     "mmsp_lse_merge": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32,
                         c_void_p], c_int32),
     "mmsp_attn_bwd": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32,
@@ -136,6 +138,13 @@ def mmsp_attn_fwd(q, k, v, N, P, Hq, Hkv, d, scale, causal, step_begin, step_end
                             int(causal), int(step_begin), int(step_end), _ptr(o_acc), _ptr(lse), _ptr(o_out),
                             int(flags), _ptr(doc_start), _stream(stream))
     return _check("mmsp_attn_fwd", rc)
+
+
+def mmsp_shard_rope(src, dst, N, P, H, d, theta=1e7, interleaved=False, doc_start=None, inverse=False, stream=None):
+    """Shard gather with RoPE applied (or the transposed scatter; see mmsp.h)."""
+    rc = _lib.mmsp_shard_rope(_ptr(src), _ptr(dst), int(N), int(P), int(H), int(d), float(theta),
+                              int(bool(interleaved)), _ptr(doc_start), int(bool(inverse)), _stream(stream))
+    return _check("mmsp_shard_rope", rc)
 
 
 def mmsp_doc_starts(doc_len, N, doc_start, stream=None):

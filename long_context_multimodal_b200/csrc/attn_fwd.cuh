@@ -48,7 +48,14 @@ namespace fwd {
 constexpr int BM = 128;      // query rows per tile
 constexpr int BN = 128;      // keys per tile
 constexpr int NSTAGE = 5;    // K/V ring stages
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;  // three warpgroups: TMA + MMA (+2 idle warps), softmax A, softmax B
+// Register split: the launch gives 168 per thread (384 x 168 <= 65,536);
+// the control warpgroup drops to kRegCtl and the softmax warpgroups rise to
+// kRegSoftmax, keeping 128 x kRegCtl + 256 x kRegSoftmax <= 384 x 168.
+constexpr int kRegLaunch = 168;
+constexpr int kRegCtl = 104;
+constexpr int kRegSoftmax = 192;
+static_assert(128 * kRegCtl + 256 * kRegSoftmax <= kThreads * kRegLaunch, "register split exceeds the launch");
 constexpr int HALF = 128 * 128;  // bytes of one 128-row x 64-column bf16 half tile
 
 struct Params {
@@ -257,7 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const long long cap = p.wait_cap;
-
+  if (warp < 4) {
+  setmaxnreg_dec<kRegCtl>();
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     // The whole warp runs the (uniform) control flow; lane 0 issues.
@@ -313,49 +321,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idO = idesc_bf16_f32(BM, D, 0, 1);
       const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
       const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
-      const uint32_t sQ[2] = {sQ0, sQ1};
+      // operand descriptors, computed once: Q tiles, and stage 0 of the K/V
+      // ring (stage s is (s * KT) >> 4 further)
+      const uint64_t dQ[2] = {desc_kmajor_sw128(sQ0), desc_kmajor_sw128(sQ1)};
+      const uint64_t dK0 = desc_kmajor_sw128(sKV);
+      const uint64_t dV0 = desc_mnmajor_sw128(sKV, HALF);
       const std::integral_constant<int, 0> kA{};
       const std::integral_constant<int, 1> kB{};
-      int64_t pos = 0;
+      uint32_t pos = 0;  // K/V ring position (stage pos % NSTAGE)
       uint32_t qcnt = 0;
       uint32_t s_cnt[2] = {0, 0}, pv_cnt[2] = {0, 0}, epi_cnt[2] = {0, 0};
 
-      auto wait_full = [&](int64_t ps) {
-        mbar_wait(kv_full((int)(ps % NSTAGE)), (uint32_t)((ps / NSTAGE) & 1), abort_flag, cap);
+      auto wait_full = [&](uint32_t ps) {
+        mbar_wait(kv_full((int)(ps % NSTAGE)), (ps / NSTAGE) & 1, abort_flag, cap);
         tc_fence_after();
       };
       bool first_pv[2] = {true, true};
-      auto issue_S = [&](auto X, int64_t kpos) {
+      // Waits and issues are split so that all of a group's waits (P ready,
+      // O free, S buffer free) come before its PV and next S, which then go
+      // to the tensor pipe back to back.
+      auto wait_s_free = [&](auto X) {  // the softmax has released S_X
         constexpr int x = decltype(X)::value;
-        if (s_cnt[x] > 0) {
-          mbar_wait(s_free(x), (s_cnt[x] - 1) & 1, abort_flag, cap);
-          tc_fence_after();
-        }
-        const uint32_t sk = sKV + (uint32_t)(kpos % NSTAGE) * L::KT;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
-          mma_bf16_ss_w(leader, tS[x], desc_kmajor_sw128(sQ[x] + off), desc_kmajor_sw128(sk + off), idS, kk > 0 ? 1u : 0u);
-        }
-        mma_commit_w(leader, s_full(x));
-        ++s_cnt[x];
+        if (s_cnt[x] > 0) mbar_wait(s_free(x), (s_cnt[x] - 1) & 1, abort_flag, cap);
       };
-      auto issue_PV = [&](auto X, int64_t vpos) {
+      auto wait_p = [&](auto X) {  // P_X written; O_X free at an item's first PV
         constexpr int x = decltype(X)::value;
         mbar_wait(p_full(x), pv_cnt[x] & 1, abort_flag, cap);
-        tc_fence_after();
-        if (first_pv[x] && epi_cnt[x] > 0) {
-          mbar_wait(o_free(x), (epi_cnt[x] - 1) & 1, abort_flag, cap);
-          tc_fence_after();
+        if (first_pv[x] && epi_cnt[x] > 0) mbar_wait(o_free(x), (epi_cnt[x] - 1) & 1, abort_flag, cap);
+      };
+      auto mma_S = [&](auto X, uint32_t kpos) {  // S_X = Q_X K^T
+        constexpr int x = decltype(X)::value;
+        const uint64_t dk = dK0 + (uint64_t)((kpos % NSTAGE) * (L::KT >> 4));
+        if (leader) {
+          mma_ss_kblock<D / 16, HALF>(tS[x], dQ[x], dk, idS, 0u);
+          mma_commit(s_full(x));
         }
-        const uint32_t sv = sKV + (uint32_t)(vpos % NSTAGE) * L::KT;
+        ++s_cnt[x];
+      };
+      auto mma_PV = [&](auto X, uint32_t vpos) {  // O_X += P_X V
+        constexpr int x = decltype(X)::value;
+        const uint64_t dv = dV0 + (uint64_t)((vpos % NSTAGE) * (L::KT >> 4));
         // P_X is in TMEM over the first 64 columns of S_X (8 columns = 16
         // keys per instruction)
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_bf16_ts_w(leader, tO[x], tS[x] + 8u * kk, desc_mnmajor_sw128(sv + kk * 2048, HALF), idO,
-                        (kk > 0 || !first_pv[x]) ? 1u : 0u);
-        mma_commit_w(leader, o_done(x));
+        if (leader) {
+          mma_ts_kblock<BN / 16>(tO[x], tS[x], dv, idO, first_pv[x] ? 0u : 1u);
+          mma_commit(o_done(x));
+        }
         ++pv_cnt[x];
         first_pv[x] = false;
       };
@@ -369,28 +380,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         TileIter<DOC> ti(p, it);
         bool has = ti.next();
         if (has) {
-          const int64_t kpos = pos++;
+          const uint32_t kpos = pos++;
           wait_full(kpos);
-          if (ti.actA) issue_S(kA, kpos);
-          if (ti.actB) issue_S(kB, kpos);
+          if (ti.actA) wait_s_free(kA);
+          if (ti.actB) wait_s_free(kB);
+          tc_fence_after();
+          if (ti.actA) mma_S(kA, kpos);
+          if (ti.actB) mma_S(kB, kpos);
           mma_commit_w(leader, kv_empty((int)(kpos % NSTAGE)));
         }
         while (has) {
           const bool curA = ti.actA, curB = ti.actB;
-          const int64_t vpos = pos++;
+          const uint32_t vpos = pos++;
           wait_full(vpos);
+          // next tile's bookkeeping and K wait first, so that S_X of the
+          // next tile follows PV_X in the tensor pipe without a gap
           const bool has_next = ti.next();
-          int64_t kn = -1;
-          if (curA) issue_PV(kA, vpos);
+          uint32_t kn = 0;
           if (has_next) {
             kn = pos++;
             wait_full(kn);
-            if (ti.actA) issue_S(kA, kn);
           }
-          if (curB) issue_PV(kB, vpos);
+          const bool nA = has_next && ti.actA, nB = has_next && ti.actB;
+          if (curA || nA) {
+            if (curA) wait_p(kA);
+            if (nA) wait_s_free(kA);
+            tc_fence_after();
+            if (curA) mma_PV(kA, vpos);
+            if (nA) mma_S(kA, kn);
+          }
+          if (curB || nB) {
+            if (curB) wait_p(kB);
+            if (nB) wait_s_free(kB);
+            tc_fence_after();
+            if (curB) mma_PV(kB, vpos);
+          }
           mma_commit_w(leader, kv_empty((int)(vpos % NSTAGE)));
           if (has_next) {
-            if (ti.actB) issue_S(kB, kn);
+            if (nB) mma_S(kB, kn);
             mma_commit_w(leader, kv_empty((int)(kn % NSTAGE)));
           }
           has = has_next;
@@ -400,9 +427,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!first_pv[1]) ++epi_cnt[1];
       }
     }
+  }
   } else {
+  setmaxnreg_inc<kRegSoftmax>();
+  {
     // --------------------------------------------------- softmax groups
-    const int grp = (warp - 2) >> 2;  // 0: tile A, 1: tile B
+    const int grp = (warp - 4) >> 2;  // 0: tile A, 1: tile B
     const int wq = warp & 3;           // TMEM lane quarter this warp may access
     const int row = wq * 32 + lane;    // row of the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
@@ -438,31 +468,38 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (DOC) lb = lo_row - ti.kglob0;
         }
-        // pass 1: row max over the tile, 64 columns per TMEM round trip
         // The per-tile softmax, compiled twice: with the causal / ragged-tail
-        // mask (diagonal and last tiles) and without it (all other tiles).
+        // / document mask (diagonal, last and boundary tiles) and without it.
+        // One TMEM read per tile: the thread's whole row of S (128 fp32)
+        // stays in registers for the max and the exponentials.
         float alpha = 1.f, rs = 0.f;
         bool need = false;
         auto tile = [&](auto MKc) {
           constexpr bool MK = decltype(MKc)::value;
-          // eight independent max chains instead of one 128-long chain
-          float mxv[8];
+          uint32_t sr[128];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) mxv[u] = -CUDART_INF_F;
+          for (int c = 0; c < 4; ++c)
+            tmem_ld32(tS + 32u * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+          tmem_wait_ld();
+          if (MK) {  // masked columns become -inf: their exponential is 0
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t sr[64];
-            tmem_ld32(tS + 64u * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-            tmem_ld32(tS + 64u * h + 32u, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 64; ++j) {
-              const float x = (!MK || (64 * h + j < lim && 64 * h + j >= lb)) ? __uint_as_float(sr[j]) : -CUDART_INF_F;
-              mxv[j & 7] = fmaxf(mxv[j & 7], x);
-            }
+            for (int j = 0; j < 128; ++j)
+              if (!(j < lim && j >= lb)) sr[j] = 0xff800000u;
           }
-          const float mx = fmaxf(fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])),
-                                 fmaxf(fmaxf(mxv[4], mxv[5]), fmaxf(mxv[6], mxv[7])));
+          // row max: four independent chains of three-input maxima over
+          // columns 0-3 (seeds), 4-123 (15 rounds of 8) and 124-127
+          float mxv[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) mxv[u] = __uint_as_float(sr[u]);
+#pragma unroll
+          for (int j = 4; j < 124; j += 8) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              mxv[u] = max3f(mxv[u], __uint_as_float(sr[j + 2 * u]), __uint_as_float(sr[j + 2 * u + 1]));
+          }
+          mxv[0] = max3f(mxv[0], __uint_as_float(sr[124]), __uint_as_float(sr[125]));
+          mxv[1] = max3f(mxv[1], __uint_as_float(sr[126]), __uint_as_float(sr[127]));
+          const float mx = max3f(mxv[0], mxv[1], fmaxf(mxv[2], mxv[3]));
           const float mc = fmaxf(m, mx * sl2);
           need = mc > m + 8.0f;
           alpha = 1.f;
@@ -478,40 +515,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(o_done(grp), (pv_cnt - 1) & 1, abort_flag, cap);
             tc_fence_after();
           }
-          // pass 2: P = 2^(s*scale*log2e - m) as bf16 pairs written back into
-          // TMEM over columns of S this thread has already read (half h of the
-          // keys lands in columns [32h, 32h+32)); the PV MMA reads it there.
-          float rsv[8];  // eight independent partial row sums
+          // P = 2^(s*scale*log2e - m) as bf16 pairs written back into TMEM
+          // over the first 64 columns of S (key pair u in column u); the PV
+          // MMA reads it there. Scale-and-shift and the row sums run as
+          // packed fp32 pairs.
+          const float2 sl2v = make_float2(sl2, sl2), nmu = make_float2(-mu, -mu);
+          float2 rsv[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                           make_float2(0.f, 0.f)};
 #pragma unroll
-          for (int u = 0; u < 8; ++u) rsv[u] = 0.f;
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t pk[32];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t sr[64];
-            tmem_ld32(tS + 64u * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-            tmem_ld32(tS + 64u * h + 32u, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-            tmem_wait_ld();
-#pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-              uint32_t pk[16];
-#pragma unroll
-              for (int u = 0; u < 16; ++u) {
-                const int j0 = 32 * q2 + 2 * u;
-                float e0 = ex2_approx(fmaf(__uint_as_float(sr[j0]), sl2, -mu));
-                float e1 = ex2_approx(fmaf(__uint_as_float(sr[j0 + 1]), sl2, -mu));
-                if (MK && (64 * h + j0 >= lim || 64 * h + j0 < lb)) e0 = 0.f;
-                if (MK && (64 * h + j0 + 1 >= lim || 64 * h + j0 + 1 < lb)) e1 = 0.f;
-                rsv[(2 * u) & 7] += e0;
-                rsv[(2 * u + 1) & 7] += e1;
-                pk[u] = pack_bf16x2_alu(e0, e1);
-              }
-              tmem_st16(tS + 32u * h + 16u * q2, pk);
+            for (int u = 0; u < 32; ++u) {
+              const int j0 = 64 * hh + 2 * u;
+              const float2 x =
+                  fma_f32x2(make_float2(__uint_as_float(sr[j0]), __uint_as_float(sr[j0 + 1])), sl2v, nmu);
+              const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+              rsv[u & 3] = add_f32x2(rsv[u & 3], e);
+              pk[u] = pack_bf16x2_alu(e.x, e.y);
             }
+            tmem_st32(tS + 32u * hh, pk);
           }
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(s_free(grp));
-          rs = ((rsv[0] + rsv[1]) + (rsv[2] + rsv[3])) + ((rsv[4] + rsv[5]) + (rsv[6] + rsv[7]));
+          const float2 r01 = add_f32x2(rsv[0], rsv[1]), r23 = add_f32x2(rsv[2], rsv[3]);
+          const float2 r = add_f32x2(r01, r23);
+          rs = r.x + r.y;
         };
         if (msk) tile(std::true_type{});
         else tile(std::false_type{});
@@ -611,6 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(o_free(grp));
       }
     }
+  }
   }
 
   tc_fence_before();

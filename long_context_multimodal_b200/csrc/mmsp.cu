@@ -19,6 +19,7 @@
 #include "merge.cuh"
 #include "attn_fwd.cuh"
 #include "attn_bwd.cuh"
+#include "rope.cuh"
 
 using namespace mmsp;
 
@@ -229,6 +230,51 @@ int mmsp_doc_starts(const int32_t* doc_len, int32_t n_doc, int64_t N, int32_t* d
   return ok();
 }
 
+int mmsp_shard_rope(const void* src, void* dst, int64_t N, int32_t P, int32_t H, int32_t d, double theta,
+                    int32_t interleaved, const int32_t* doc_start, int32_t inverse, void* stream) {
+  int rc = check_common(N, P);
+  if (rc) return rc;
+  if (H < 1) return fail(MMSP_EINVAL, "H must be >= 1");
+  if (!(d == 8 || d == 16 || d == 32 || d == 64 || d == 128 || d == 256))
+    return fail(MMSP_EINVAL, "d must be one of 8, 16, 32, 64, 128, 256 (got %d)", d);
+  if (!(theta > 1.0) || !std::isfinite(theta)) return fail(MMSP_EINVAL, "theta must be finite and > 1");
+  if (interleaved != 0 && interleaved != 1) return fail(MMSP_EINVAL, "interleaved must be 0 or 1");
+  if (inverse != 0 && inverse != 1) return fail(MMSP_EINVAL, "inverse must be 0 or 1");
+  if (!src || !dst) return fail(MMSP_EINVAL, "src and dst must be non-NULL");
+  if (!aligned16(src) || !aligned16(dst)) return fail(MMSP_EINVAL, "src and dst must be 16-byte aligned");
+  if (doc_start && ((uintptr_t)doc_start & 3u)) return fail(MMSP_EINVAL, "doc_start must be 4-byte aligned");
+  const int64_t bytes = N * (int64_t)H * d * 2;
+  const char* s0 = static_cast<const char*>(src);
+  const char* d0 = static_cast<const char*>(dst);
+  if (s0 < d0 + bytes && d0 < s0 + bytes) return fail(MMSP_EINVAL, "src and dst overlap");
+  if (N == 0) return ok();
+  int dev, sms;
+  if ((rc = current_device(&dev)) || (rc = device_sms(dev, &sms))) return rc;
+  RopeParams rp;
+  for (int i = 0; i < kRopeMaxPairs; ++i) rp.inv_freq[i] = i < d / 2 ? std::pow(theta, -2.0 * i / d) : 0.0;
+  rp.N = (int32_t)N;
+  rp.P = P;
+  rp.H = H;
+  rp.inverse = inverse;
+  rp.doc_start = doc_start;
+  int64_t blocks = (N + 7) / 8;  // 8 warps (rows) per block
+  if (blocks > 16LL * sms) blocks = 16LL * sms;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const __nv_bfloat16* sb = static_cast<const __nv_bfloat16*>(src);
+  __nv_bfloat16* db = static_cast<__nv_bfloat16*>(dst);
+#define MMSP_ROPE(DD)                                                                            \
+  case DD:                                                                                       \
+    if (interleaved)                                                                             \
+      shard_rope_kernel<DD, true><<<(unsigned)blocks, 256, 0, st>>>(rp, sb, db);                 \
+    else                                                                                         \
+      shard_rope_kernel<DD, false><<<(unsigned)blocks, 256, 0, st>>>(rp, sb, db);                \
+    break;
+  switch (d) { MMSP_ROPE(8) MMSP_ROPE(16) MMSP_ROPE(32) MMSP_ROPE(64) MMSP_ROPE(128) MMSP_ROPE(256) }
+#undef MMSP_ROPE
+  MMSP_CUDA(cudaGetLastError());
+  return ok();
+}
+
 int mmsp_lse_merge(const float* o_a, const float* lse_a, const float* o_b, const float* lse_b, float* o_out,
                    float* lse_out, int64_t rows, int32_t H, int32_t d, void* stream) {
   if (rows < 0 || H < 1) return fail(MMSP_EINVAL, "rows must be >= 0 and H >= 1");
@@ -265,6 +311,13 @@ int launch_fwd(int dev, int vi, int64_t grid, cudaStream_t st, const CUtensorMap
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_dev[dev].fwd_attr[vi]) {
+      // The kernel's warpgroups re-split the launch's registers; a build
+      // that launches with fewer per thread would make the split wait.
+      cudaFuncAttributes fa;
+      MMSP_CUDA(cudaFuncGetAttributes(&fa, fwd::attn_fwd_kernel<D, DOC>));
+      if (fa.numRegs < fwd::kRegLaunch)
+        return fail(MMSP_ECUDA, "forward kernel built with %d registers per thread, the register split needs %d",
+                    fa.numRegs, fwd::kRegLaunch);
       MMSP_CUDA(cudaFuncSetAttribute(fwd::attn_fwd_kernel<D, DOC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      fwd::Smem<D>::ALLOC));
       g_dev[dev].fwd_attr[vi] = true;

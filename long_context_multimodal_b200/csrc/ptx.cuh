@@ -171,6 +171,49 @@ __device__ __forceinline__ void mma_bf16_ts_w(uint32_t leader, uint32_t d_tmem, 
   if (leader) mma_bf16_ts(d_tmem, a_tmem, bdesc, idesc, accumulate);
 }
 
+// A run of NK tcgen05.mma steps along K issued back to back by the calling
+// thread (call it from one elected thread). The operand descriptors are
+// computed once by the caller and advanced by compile-time constants: a
+// descriptor's start-address field holds the shared address in 16-byte
+// units, so adding (bytes >> 4) to the descriptor moves it, as long as the
+// address stays below 256 KB (every shared address does). Only the first
+// step honours `accumulate`; the rest accumulate.
+//
+// SS form, both operands K-major SWIZZLE_128B tiles stored as 64-element
+// (128-byte) column halves `half_bytes` apart: step kk reads 16 elements at
+// byte (kk / 4) * half_bytes + (kk % 4) * 32 of each operand.
+template <int NK, uint32_t HALF_BYTES>
+__device__ __forceinline__ void mma_ss_kblock(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < NK; ++kk) {
+    const uint64_t off = (uint64_t)((kk >> 2) * (HALF_BYTES >> 4) + (kk & 3) * 2);
+    mma_bf16_ss(d_tmem, adesc + off, bdesc + off, idesc, kk ? 1u : accumulate);
+  }
+}
+
+// SS form with A K-major (as above) and B MN-major: step kk reads rows
+// [16 kk, 16 kk + 16) of B, 16 * 128 bytes further each step.
+template <int NK, uint32_t HALF_BYTES>
+__device__ __forceinline__ void mma_ss_kblock_bmn(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                  uint32_t accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < NK; ++kk) {
+    const uint64_t aoff = (uint64_t)((kk >> 2) * (HALF_BYTES >> 4) + (kk & 3) * 2);
+    mma_bf16_ss(d_tmem, adesc + aoff, bdesc + (uint64_t)(kk * 128), idesc, kk ? 1u : accumulate);
+  }
+}
+
+// TS form: A from tensor memory (8 columns = 16 bf16 per step), B MN-major
+// (16 rows of 128 bytes per step).
+template <int NK>
+__device__ __forceinline__ void mma_ts_kblock(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < NK; ++kk)
+    mma_bf16_ts(d_tmem, a_tmem + 8u * kk, bdesc + (uint64_t)(kk * 128), idesc, kk ? 1u : accumulate);
+}
+
 // One arrival on `bar` once every tcgen05 async op issued so far by this
 // thread has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -263,6 +306,47 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Per-warpgroup register budget (all four warps of a warpgroup execute the
+// same call). The launch's registers (threads x registers per thread) bound
+// the sum over warpgroups.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed fp32 pair arithmetic (one instruction for two lanes of work on
+// sm_100): d = a * b + c and d = a + b, element-wise, round to nearest.
+__device__ __forceinline__ float2 fma_f32x2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 add_f32x2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
 }
 
 // Two floats to a bf16 pair (lo in the low half), rounded to nearest with
