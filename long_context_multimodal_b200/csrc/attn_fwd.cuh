@@ -53,8 +53,8 @@ constexpr int kThreads = 384;  // three warpgroups: TMA + MMA (+2 idle warps), s
 // the control warpgroup drops to kRegCtl and the softmax warpgroups rise to
 // kRegSoftmax, keeping 128 x kRegCtl + 256 x kRegSoftmax <= 384 x 168.
 constexpr int kRegLaunch = 168;
-constexpr int kRegCtl = 104;
-constexpr int kRegSoftmax = 192;
+constexpr int kRegCtl = 120;
+constexpr int kRegSoftmax = 176;
 static_assert(128 * kRegCtl + 256 * kRegSoftmax <= kThreads * kRegLaunch, "register split exceeds the launch");
 constexpr int HALF = 128 * 128;  // bytes of one 128-row x 64-column bf16 half tile
 
