@@ -18,7 +18,7 @@
 // The CTA visits the item's K/V tiles of 128 keys in ring order and skips
 // (chunk, tile) pairs the causal mask empties.
 //
-// Warp roles (320 threads, one CTA per SM):
+// Warp roles (384 threads = three warpgroups, one CTA per SM):
 //   warp 0      TMA producer: Q tiles A/B once per item, then K_j, V_j into
 //               a 5-stage ring of 128 x d bf16 tiles (128-byte swizzle).
 //   warp 1      MMA issuer (warp-uniform, one lane issues): S_X = Q_X K_j^T
@@ -28,10 +28,14 @@
 //               tensor core works on one tile while the softmax warps work
 //               on the other. tcgen05 MMAs of one thread run in issue order,
 //               so S_X(j+1) overwrites P_X(j) only after PV_X(j) read it.
-//   warps 2-5   softmax for tile A, warps 6-9 for tile B: one thread per row
-//               (TMEM lane), fp32 online softmax in base 2, P written to
-//               TMEM as bf16, lazy O rescale (only when the running max grows
-//               by more than 2^8), epilogue O / l and LSE.
+//   warps 2-3   idle (they complete the first warpgroup's register release).
+//   warps 4-7   softmax for tile A, warps 8-11 for tile B: one thread per
+//               row (TMEM lane) holding its whole row of S in registers,
+//               fp32 online softmax in base 2, P written to TMEM as bf16,
+//               lazy O rescale (only when the running max grows by more than
+//               2^8), epilogue O / l and LSE.
+// The first warpgroup gives registers to the two softmax warpgroups
+// (setmaxnreg), see kRegCtl / kRegSoftmax.
 // TMEM: S_A [0,128) S_B [128,256) O_A [256,256+d) O_B [256+d,256+2d).
 #pragma once
 
