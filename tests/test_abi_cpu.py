@@ -98,3 +98,32 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     mod = importlib.util.module_from_spec(spec)
     with pytest.raises(ImportError):
         spec.loader.exec_module(mod)
+
+
+def test_documents_and_rope_reject_bad_arguments():
+    import long_context_multimodal_b200 as m
+
+    p = 1 << 20
+    # document starts: table must be valid and sum to N
+    _einval(m.mmsp_doc_starts, [4, 4], 16, p)                     # sums to 8, not 16
+    _einval(m.mmsp_doc_starts, [8, 0, 8], 16, p)                  # empty document
+    _einval(m.mmsp_doc_starts, [16], 16, p + 2)                   # misaligned output
+    _einval(m.mmsp_doc_starts, np.ones(4097, np.int32), 4097, p)  # over capacity
+    # doc_start on the attention calls needs causal attention and alignment
+    ok = dict(q=p, k=p, v=p, N=4096, P=4, Hq=4, Hkv=4, d=64, scale=0.125, causal=1, step_begin=0, step_end=4,
+              o_acc=p, lse=p, o_out=p, flags=m.MMSP_FINALIZE)
+    _einval(m.mmsp_attn_fwd, **dict(ok, causal=0), doc_start=p)
+    _einval(m.mmsp_attn_fwd, **ok, doc_start=p + 2)
+    ws = m.mmsp_bwd_workspace_bytes(4096, 4, 4, 128)
+    _einval(m.mmsp_attn_bwd, p, p, p, p, p, p, 4096, 4, 4, 4, 128, 0.088, 0, p, p, p, None, p, ws, doc_start=p)
+    # RoPE gather: head size, base, flags, alignment, overlap, sharding
+    R = m.mmsp_shard_rope
+    _einval(R, p, p + (1 << 24), 64, 2, 2, 48)                    # d not supported
+    _einval(R, p, p + (1 << 24), 64, 2, 2, 512)
+    _einval(R, p, p + (1 << 24), 64, 2, 2, 64, theta=1.0)         # base must exceed 1
+    _einval(R, p, p + (1 << 24), 64, 2, 2, 64, theta=float("nan"))
+    _einval(R, p, p + (1 << 24), 64, 3, 2, 64)                    # N % 2P
+    _einval(R, p, p + (1 << 24), 64, 2, 0, 64)                    # no heads
+    _einval(R, p + 8, p + (1 << 24), 64, 2, 2, 64)                # misaligned
+    _einval(R, p, p + 64, 64, 2, 2, 64)                           # overlapping rows
+    _einval(R, p, p + (1 << 24), 64, 2, 2, 64, doc_start=p + 1)   # misaligned document starts
