@@ -101,3 +101,23 @@ def test_workload_layouts(name):
     assert int(sl[sk == mi.TEXT].sum()) == w.text_tokens
     assert np.all(sl >= 1)
     assert sk[0] == mi.TEXT  # the sequence opens with text
+
+
+@pytest.mark.parametrize("N,seed", [(1000, 5), (4608, 3), (65536, 44), (7, 1)])
+def test_packed_documents_recipe(N, seed):
+    """The packed-video input recipe: documents of (prompt text, whole
+    576-token frames, answer text), cut at N; the segment table covers the
+    same tokens and only the last document may hold a partial frame."""
+    doc_len, seg_len, seg_kind = mi.packed_documents(N, seed)
+    assert int(doc_len.sum()) == N and int(seg_len.sum()) == N
+    assert (doc_len >= 1).all() and (seg_len >= 1).all()
+    kinds = mi.token_kinds(seg_len, seg_kind)
+    starts = np.concatenate([[0], np.cumsum(doc_len)[:-1]])
+    for i, (s0, L) in enumerate(zip(starts, doc_len)):
+        k = kinds[s0:s0 + L]
+        assert k[0] == mi.TEXT  # every document opens with its prompt
+        if i < len(doc_len) - 1:
+            # frames are whole inside complete documents
+            vis = np.flatnonzero(np.diff(np.concatenate([[0], k.astype(np.int8), [0]])))
+            runs = vis[1::2] - vis[0::2]
+            assert (runs % mi.FRAME_TOKENS == 0).all()
