@@ -12,6 +12,11 @@
  * 1/sqrt(head_dim), per-step block attention). The log-sum-exp combine, the
  * causal mask, zigzag sharding and GQA head grouping are readings of those
  * passages (the page's sketch sums separately normalised blocks).
+ * Extensions on the same path: packed documents with the attention mask
+ * reset at each document (section "Critical Operational Best Practices",
+ * dynamic sequence packing; mmsp_doc_starts and the doc_start arguments),
+ * and the rotary position embedding with base 10^7 fused into the shard
+ * gather (three-stage curriculum, Stage 2; mmsp_shard_rope).
  *
  * Conventions for every entry point
  *   - Returns an mmsp_status; MMSP_OK on success. On failure the message of
