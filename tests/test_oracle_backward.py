@@ -117,3 +117,27 @@ def test_document_sampled_helpers_agree_with_whole_backward():
     kk = A.attention_bwd_keys(q[70:], k, v, do[70:], keys, block=9, doc_start=ds)
     np.testing.assert_allclose(kk["dK"], g["dK"][keys], atol=1e-12)
     np.testing.assert_allclose(kk["dV"], g["dV"][keys], atol=1e-12)
+
+
+@pytest.mark.parametrize("lengths,hq,hkv,d", [([9, 20, 1, 14], 4, 2, 8), ([1, 1, 40, 3, 19], 6, 3, 16)])
+def test_document_mask_matches_torch_sdpa_autograd_fp64(lengths, hq, hkv, d):
+    """Library cross-check of the document-masked forward and backward:
+    torch scaled_dot_product_attention with an explicit boolean mask
+    (doc_start[i] <= j <= i) and autograd, in fp64 on CPU."""
+    N = sum(lengths)
+    q, k, v, do = _inputs(N, hq, hkv, d, 31 + N)
+    ds = A.document_starts(lengths)
+    g = A.causal_attention_bwd(q, k, v, do, block=8, doc_start=ds)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    G = hq // hkv
+    i = torch.arange(N)[:, None]
+    j = torch.arange(N)[None, :]
+    mask = (j <= i) & (j >= torch.as_tensor(ds)[:, None])
+    out = torch.nn.functional.scaled_dot_product_attention(
+        tq.transpose(0, 1), tk.repeat_interleave(G, 1).transpose(0, 1),
+        tv.repeat_interleave(G, 1).transpose(0, 1), attn_mask=mask).transpose(0, 1)
+    out.backward(torch.tensor(do))
+    np.testing.assert_allclose(g["O"], out.detach().numpy(), atol=1e-12)
+    np.testing.assert_allclose(g["dQ"], tq.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(g["dK"], tk.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(g["dV"], tv.grad.numpy(), atol=1e-11)
