@@ -286,6 +286,26 @@ class Path:
                          stream=stream)
 
 
+def document_forward(m, path, w, dev, stream, time_calls):
+    """Forward of the packed-document variant: the workload's N tokens as a
+    buffer of short videos (mmsp_inputs.packed_documents), every document's
+    attention causal and isolated. Algorithmic flops count the visible
+    pairs, 4 d Hq sum_docs L (L + 1) / 2."""
+    import torch
+
+    doc_len, _, _ = mi.packed_documents(w.N, 3000 + w.index)
+    ds = torch.empty(w.N, dtype=torch.int32, device=dev)
+    m.mmsp_doc_starts(doc_len, w.N, ds, stream=stream)
+    L = doc_len.astype(np.float64)
+    flops = 4.0 * w.d * w.hq * float((L * (L + 1) / 2).sum())
+    ms = time_calls(lambda: m.mmsp_attn_fwd(path.ql, path.kl, path.vl, w.N, w.P, w.hq, w.hkv, w.d, path.scale, 1, 0,
+                                            w.P, None, path.lse, path.ol, m.MMSP_FINALIZE, doc_start=ds,
+                                            stream=stream))
+    m.mmsp_device_status(stream)
+    return {"documents": int(doc_len.size), "mean_tokens": float(L.mean()), "ms": ms,
+            "algorithmic_flops": flops, "tflops": flops / (ms * 1e-3) / 1e12}
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -426,6 +446,14 @@ def run_gpu(args):
             line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                                     "sample": f"{args.ref_rows} random query rows x {w.hq} heads of {w.name}: "
                                               f"fp64 forward + dQ backward ({dt:.1f} s)"}
+        if ws == 1:
+            # packed documents (attention reset per document) over the same
+            # rank-local Q, K, V; measured last and guarded so that a problem
+            # here is reported in the line instead of losing it
+            try:
+                line["document_masked_fwd"] = document_forward(m, path, w, dev, stream, time_calls)
+            except Exception as exc:  # noqa: BLE001
+                line["document_masked_fwd"] = {"error": f"{type(exc).__name__}: {exc}"}
         print(json.dumps(line), flush=True)
     if ws > 1:
         dist.barrier()
