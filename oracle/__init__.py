@@ -17,7 +17,7 @@ Sources ("page" = the web page the method is described on):
   (B,S,H,D) layout) and class ``LongVILAParallelContext`` (ring neighbours:
   receive from the previous ring rank, send to the next).
 
-Readings where the pages are silent or wrong (each also listed in the design doc):
+Readings where the pages are silent or wrong:
 the partial results of the ring steps are combined with the log-sum-exp merge
 (the page's sketch sums separately normalised blocks, which is not attention);
 the causal mask is j <= i over global positions; zigzag sharding gives rank r

@@ -67,35 +67,51 @@ def document_starts(doc_len):
     return np.asarray(out, np.int64)
 
 
-def _visible(jmax, rows, lo):
-    """[R, jmax] mask: key j visible to row i iff lo_i <= j <= i (lo_i = 0
-    without documents)."""
-    rows_t = torch.as_tensor(np.asarray(rows, np.int64))
-    j = torch.arange(jmax)[None, :]
-    vis = j <= rows_t[:, None]
+def _scores(qr, rows, K, scale, lo=None):
+    """s_ij = (q_i . k_j) * scale for the keys K[:jmax] (fp64 torch), with
+    -inf where key j is not visible to the row: j > i (causal), or j < lo_i
+    (before the row's document start). qr is [R, d]; rows [R] holds each
+    vector's global position (rows may repeat when several heads of one
+    position are stacked). Columns before min(rows) + 1 are visible to every
+    row and columns from max(lo) on pass the document test, so the mask is
+    only applied where it can remove a key."""
+    jmax = K.shape[0]
+    s = qr @ K.T
+    s.mul_(scale)
+    rows = np.asarray(rows, np.int64)
+    j_first = int(rows.min()) + 1
+    if j_first < jmax:
+        s[:, j_first:].masked_fill_(torch.arange(j_first, jmax)[None, :] > torch.as_tensor(rows)[:, None], NEG_INF)
     if lo is not None:
-        vis &= j >= torch.as_tensor(np.asarray(lo, np.int64))[:, None]
-    return vis
+        lo = np.asarray(lo, np.int64)
+        j_last = int(lo.max())
+        if j_last > 0:
+            s[:, :j_last].masked_fill_(torch.arange(j_last)[None, :] < torch.as_tensor(lo)[:, None], NEG_INF)
+    return s
+
+
+def _softmax_rows(qr, rows, K, V, scale, lo=None):
+    """Row softmax of the visible scores and the output: returns (P, O, LSE)
+    with P_ij = exp(s_ij - m_i) / l_i, l_i = sum_j exp(s_ij - m_i),
+    m_i = max_j s_ij, O = P V and LSE_i = m_i + ln l_i. fp64 torch."""
+    p = _scores(qr, rows, K, scale, lo)
+    m = p.max(dim=1).values
+    p.sub_(m[:, None]).exp_()                                    # 0 where masked
+    l = p.sum(dim=1)
+    p.div_(l[:, None])
+    return p, p @ V, m + torch.log(l)
 
 
 def _rows_forward(qr, rows, K, V, scale, lo=None):
     """O and LSE for query vectors qr [R,d] at global positions rows [R]
     against keys K[:i+1], V[:i+1] (one head); with `lo`, only keys
-    j >= lo_i of the row's own document. Plain formula in fp64 torch CPU ops
-    (multi-threaded; same arithmetic as numpy)."""
+    j >= lo_i of the row's own document."""
     R = len(rows)
     d = V.shape[1]
     if R == 0:
         return np.zeros((R, d)), np.full(R, NEG_INF)
     jmax = int(np.max(rows)) + 1
-    qr, K, V = _t(qr), _t(K[:jmax]), _t(V[:jmax])
-    s = (qr @ K.T) * scale                                       # [R, jmax]
-    visible = _visible(jmax, rows, lo)
-    s = s.masked_fill(~visible, NEG_INF)
-    m = s.max(dim=1).values
-    lse = m + torch.log(torch.exp(s - m[:, None]).sum(dim=1))
-    p = torch.exp(s - lse[:, None])                              # 0 where masked
-    O = p @ V
+    _, O, lse = _softmax_rows(_t(qr), rows, _t(K[:jmax]), _t(V[:jmax]), scale, lo)
     return O.numpy(), lse.numpy()
 
 
@@ -123,55 +139,48 @@ def causal_attention(q, k, v, scale=None, block: int = 512, doc_start=None):
     return O, LSE
 
 
-def attention_rows(q_rows, k, v, rows, scale=None, block: int = 64, doc_start=None):
+def _head_groups(hq, hkv):
+    """The query heads that read each kv head: kv head kh -> list of h."""
+    return [[h for h in range(hq) if kv_head(h, hq, hkv) == kh] for kh in range(hkv)]
+
+
+def _row_block(n_vec, jmax, budget=1 << 26):
+    """Rows per block so that a [rows * n_vec, jmax] fp64 score matrix stays
+    within `budget` elements (memory bound only)."""
+    return max(1, budget // max(1, n_vec * jmax))
+
+
+def attention_rows(q_rows, k, v, rows, scale=None, block=None, doc_start=None):
     """Forward for selected global rows only.
 
     q_rows [R,Hq,d] holds the query vectors of global positions `rows` (the
     caller gathers them, so the whole Q need not be held in fp64); k, v are
     the whole [N,Hkv,d] tensors, converted to fp64 one kv head at a time.
-    Returns (O [R,Hq,d], LSE [R,Hq]).
+    Returns (O [R,Hq,d], LSE [R,Hq]). block: rows per block (default: a
+    memory budget).
     """
-    q_rows = _f64(q_rows)
-    rows = np.asarray(rows, np.int64)
-    R, hq, d = q_rows.shape
-    hkv = k.shape[1]
-    if scale is None:
-        scale = 1.0 / math.sqrt(d)
-    jmax = int(rows.max()) + 1 if R else 0
-    O = np.zeros((R, hq, d))
-    LSE = np.zeros((R, hq))
-    for kh in range(hkv):
-        K = _f64(k[:jmax, kh])
-        V = _f64(v[:jmax, kh])
-        for h in range(hq):
-            if kv_head(h, hq, hkv) != kh:
-                continue
-            for b0 in range(0, R, block):
-                sel = np.arange(b0, min(R, b0 + block))
-                lo = None if doc_start is None else np.asarray(doc_start)[rows[sel]]
-                o, l = _rows_forward(q_rows[sel, h], rows[sel], K, V, scale, lo)
-                O[sel, h] = o
-                LSE[sel, h] = l
-    return O, LSE
+    out = attention_bwd_rows(q_rows, k, v, None, rows, scale=scale, block=block, doc_start=doc_start)
+    return out["O"], out["LSE"]
 
 
 def _rows_backward(qr, dor, rows, K, V, scale, lo=None):
     """For one head and query rows: (O, LSE, D, dQ rows, P, dS) restricted to
-    keys [0, max(rows)]; P and dS are [R, jmax]. fp64 torch CPU ops."""
-    jmax = int(np.max(rows)) + 1
-    qr, dor, K, V = _t(qr), _t(dor), _t(K[:jmax]), _t(V[:jmax])
-    s = (qr @ K.T) * scale
-    visible = _visible(jmax, rows, lo)
-    s = s.masked_fill(~visible, NEG_INF)
-    m = s.max(dim=1).values
-    lse = m + torch.log(torch.exp(s - m[:, None]).sum(dim=1))
-    p = torch.exp(s - lse[:, None])
-    o = p @ V
-    D = (dor * o).sum(dim=1)
-    dp = dor @ V.T
-    ds = p * (dp - D[:, None])
-    dq = scale * (ds @ K)
+    keys [0, max(rows)]; P and dS are [R, jmax]."""
+    o, lse, D, dq, p, ds = _rows_backward_t(_t(qr), _t(dor), rows, _t(K), _t(V), scale, lo)
     return o.numpy(), lse.numpy(), D.numpy(), dq.numpy(), p.numpy(), ds.numpy()
+
+
+def _rows_backward_t(qr, dor, rows, K, V, scale, lo=None):
+    """_rows_backward on fp64 torch tensors (K, V may hold more keys than
+    max(rows) + 1; only those are read). Returns torch tensors."""
+    jmax = int(np.max(rows)) + 1
+    K, V = K[:jmax], V[:jmax]
+    p, o, lse = _softmax_rows(qr, rows, K, V, scale, lo)
+    D = (dor * o).sum(dim=1)
+    ds = dor @ V.T                                               # dP
+    ds.sub_(D[:, None]).mul_(p)                                  # dS = P (dP - D)
+    dq = (ds @ K).mul_(scale)
+    return o, lse, D, dq, p, ds
 
 
 def causal_attention_bwd(q, k, v, do, scale=None, block: int = 512, doc_start=None):
@@ -208,44 +217,66 @@ def causal_attention_bwd(q, k, v, do, scale=None, block: int = 512, doc_start=No
     return {"O": O, "LSE": LSE, "D": Dm, "dQ": dQ, "dK": dK, "dV": dV}
 
 
-def attention_bwd_rows(q_rows, k, v, do_rows, rows, scale=None, block: int = 64, doc_start=None):
+def attention_bwd_rows(q_rows, k, v, do_rows, rows, scale=None, block=None, doc_start=None):
     """dQ (and O, LSE) for selected global rows: row i needs only keys <= i.
-    q_rows and do_rows [R,Hq,d] are the caller-gathered rows at `rows`;
-    doc_start as in causal_attention."""
-    q_rows, do_rows = _f64(q_rows), _f64(do_rows)
+    q_rows and do_rows [R,Hq,d] are the caller-gathered rows at `rows`
+    (do_rows None: forward only, no dQ); doc_start as in causal_attention.
+    The query heads that read one kv head are evaluated together (their
+    vectors stacked as rows of one matrix), in blocks of rows sorted by
+    position (`block` rows per block; default: a memory budget)."""
+    q_rows = _f64(q_rows)
     rows = np.asarray(rows, np.int64)
     R, hq, d = q_rows.shape
     hkv = k.shape[1]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    jmax = int(rows.max()) + 1 if R else 0
+    order = np.argsort(rows, kind="stable")
     dQ = np.zeros((R, hq, d))
     O = np.zeros((R, hq, d))
     LSE = np.zeros((R, hq))
-    for kh in range(hkv):
-        K = _f64(k[:jmax, kh])
-        V = _f64(v[:jmax, kh])
-        for h in range(hq):
-            if kv_head(h, hq, hkv) != kh:
-                continue
-            for b0 in range(0, R, block):
-                sel = np.arange(b0, min(R, b0 + block))
-                lo = None if doc_start is None else np.asarray(doc_start)[rows[sel]]
-                o, lse, _, dq, _, _ = _rows_backward(q_rows[sel, h], do_rows[sel, h], rows[sel], K, V, scale, lo)
-                dQ[sel, h] = dq
-                O[sel, h] = o
-                LSE[sel, h] = lse
+    if R == 0:
+        return {"O": O, "LSE": LSE, "dQ": dQ}
+    jmax_all = int(rows.max()) + 1
+    if do_rows is not None:
+        do_rows = _f64(do_rows)
+    ds_all = None if doc_start is None else np.asarray(doc_start, np.int64)
+    for kh, heads in enumerate(_head_groups(hq, hkv)):
+        G = len(heads)
+        K = _t(k[:jmax_all, kh])
+        V = _t(v[:jmax_all, kh])
+        b0 = 0
+        while b0 < R:
+            jb = int(rows[order[b0]]) + 1
+            nb = block or _row_block(G, jb)
+            sel = order[b0:b0 + nb]
+            b0 += nb
+            rr = rows[sel]
+            rep = np.repeat(rr, G)                      # position of each stacked vector
+            lo = None if ds_all is None else ds_all[rep]
+            qb = _t(q_rows[np.ix_(sel, heads)].reshape(-1, d))
+            if do_rows is None:
+                jmax = int(rr.max()) + 1
+                _, o, lse = _softmax_rows(qb, rep, K[:jmax], V[:jmax], scale, lo)
+            else:
+                dob = _t(do_rows[np.ix_(sel, heads)].reshape(-1, d))
+                o, lse, _, dq, _, _ = _rows_backward_t(qb, dob, rep, K, V, scale, lo)
+                dQ[np.ix_(sel, heads)] = dq.reshape(len(sel), G, d).numpy()
+            O[np.ix_(sel, heads)] = o.reshape(len(sel), G, d).numpy()
+            LSE[np.ix_(sel, heads)] = lse.reshape(len(sel), G).numpy()
     return {"O": O, "LSE": LSE, "dQ": dQ}
 
 
-def attention_bwd_keys(q_tail, k, v, do_tail, keys, scale=None, block: int = 64, doc_start=None):
+def attention_bwd_keys(q_tail, k, v, do_tail, keys, scale=None, block=None, doc_start=None, kv_heads=None):
     """dK and dV for selected global key positions.
 
     Key j receives contributions from rows i >= j only. q_tail and do_tail
     hold the rows [j0, N) of Q and dO, where j0 = min(keys) and N = len(k);
     those rows are computed in full (their LSE and D over keys <= i) and
     their terms are summed into the requested keys. Cheap only when the keys
-    lie near the end. doc_start as in causal_attention.
+    lie near the end. doc_start as in causal_attention. kv_heads: the kv
+    heads to compute (default all; the others stay 0). block: rows per
+    block (default: a memory budget).
+    Also returns the tail rows' O, LSE and dQ ("O_tail", ...).
     """
     keys = np.asarray(keys, np.int64)
     N = k.shape[0]
@@ -259,18 +290,39 @@ def attention_bwd_keys(q_tail, k, v, do_tail, keys, scale=None, block: int = 64,
     q_tail, do_tail = _f64(q_tail), _f64(do_tail)
     dK = np.zeros((len(keys), hkv, d))
     dV = np.zeros((len(keys), hkv, d))
-    for kh in range(hkv):
-        K = _f64(k[:, kh])
-        V = _f64(v[:, kh])
-        for h in range(hq):
-            if kv_head(h, hq, hkv) != kh:
+    T = N - j0
+    O = np.zeros((T, hq, d))
+    LSE = np.zeros((T, hq))
+    dQ = np.zeros((T, hq, d))
+    ds_all = None if doc_start is None else np.asarray(doc_start, np.int64)
+    keys_t = torch.as_tensor(keys)
+    for kh, heads in enumerate(_head_groups(hq, hkv)):
+        if kv_heads is not None and kh not in kv_heads:
+            continue
+        G = len(heads)
+        K = _t(k[:, kh])
+        V = _t(v[:, kh])
+        dKk = torch.zeros((len(keys), d), dtype=torch.float64)
+        dVk = torch.zeros((len(keys), d), dtype=torch.float64)
+        i0 = j0
+        while i0 < N:
+            nb = block or _row_block(G, N)
+            rows = np.arange(i0, min(N, i0 + nb))
+            i0 += nb
+            rep = np.repeat(rows, G)
+            lo = None if ds_all is None else ds_all[rep]
+            qb = _t(q_tail[np.ix_(rows - j0, heads)].reshape(-1, d))
+            dob = _t(do_tail[np.ix_(rows - j0, heads)].reshape(-1, d))
+            o, lse, _, dq, p, ds = _rows_backward_t(qb, dob, rep, K, V, scale, lo)
+            O[np.ix_(rows - j0, heads)] = o.reshape(len(rows), G, d).numpy()
+            LSE[np.ix_(rows - j0, heads)] = lse.reshape(len(rows), G).numpy()
+            dQ[np.ix_(rows - j0, heads)] = dq.reshape(len(rows), G, d).numpy()
+            sel = np.nonzero(keys <= rows.max())[0]
+            if len(sel) == 0:
                 continue
-            for i0 in range(j0, N, block):
-                rows = np.arange(i0, min(N, i0 + block))
-                lo = None if doc_start is None else np.asarray(doc_start)[rows]
-                _, _, _, _, p, ds = _rows_backward(q_tail[rows - j0, h], do_tail[rows - j0, h], rows, K, V, scale,
-                                                   lo)
-                sel = np.nonzero(keys <= rows.max())[0]
-                dV[sel, kh] += p[:, keys[sel]].T @ do_tail[rows - j0, h]
-                dK[sel, kh] += scale * (ds[:, keys[sel]].T @ q_tail[rows - j0, h])
-    return {"dK": dK, "dV": dV}
+            ks = keys_t[torch.as_tensor(sel)]
+            dVk[sel] += p[:, ks].T @ dob
+            dKk[sel] += scale * (ds[:, ks].T @ qb)
+        dK[:, kh] = dKk.numpy()
+        dV[:, kh] = dVk.numpy()
+    return {"dK": dK, "dV": dV, "O_tail": O, "LSE_tail": LSE, "dQ_tail": dQ}
