@@ -163,12 +163,18 @@ def oracle_sample(w, rows_count, seed, inputs=None):
     from oracle import attention as A
 
     rows, qr, kc, vc, dor = inputs if inputs is not None else cpu_sample_inputs(w, rows_count, seed)
+    torch.set_num_threads(host_cores())
     t0 = time.perf_counter()
     A.attention_bwd_rows(qr, kc, vc, dor, rows)
     dt = time.perf_counter() - t0
     # each sampled row i: forward 4*d*(i+1) flops per head, forward+backward 3.5x
     flops = 3.5 * 4.0 * w.d * w.hq * float(np.sum(rows + 1))
     return flops, dt, torch.get_num_threads()
+
+
+def host_cores():
+    """Cores this process may run on (its CPU affinity set)."""
+    return len(os.sched_getaffinity(0))
 
 
 def run_reference(args):
@@ -191,7 +197,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, args.gpus),
+        "config": workload_config(w, args.gpus, args.mode),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -199,12 +205,21 @@ def run_reference(args):
     return 0
 
 
-def workload_config(w, gpus):
+def workload_config(w, gpus, mode="split"):
+    if gpus == 1:
+        par = f"one GPU holds all {w.P} virtual ranks of the ring"
+        batch = 1
+    elif mode == "split":
+        par = (f"one sequence; its {w.P} virtual ranks split over {gpus} GPUs ({w.P // gpus} each), K/V, Q, dO and "
+               f"the prepared (LSE, D) rows all-gathered with NCCL")
+        batch = 1
+    else:
+        par = f"{gpus} independent sequences, one per GPU; all {w.P} virtual ranks on each GPU"
+        batch = gpus
     return {"workload": w.name, "N": w.N, "frames": w.frames, "frame_tokens": mi.FRAME_TOKENS,
             "text_tokens": w.text_tokens, "text_segments": w.text_segments, "Hq": w.hq, "Hkv": w.hkv, "d": w.d,
-            "P_virtual_ranks": w.P, "causal": True, "global_batch": gpus, "seq_len": w.N,
-            "parallelism": f"{gpus} independent sequence(s), one per GPU; P virtual ranks per GPU",
-            "l2": "inputs larger than L2 (Q alone is N*Hq*d*2 bytes)"}
+            "P_virtual_ranks": w.P, "causal": True, "global_batch": batch, "seq_len": w.N,
+            "parallelism": par, "l2": "inputs larger than L2 (Q alone is N*Hq*d*2 bytes)"}
 
 
 def max_over_ranks(values, ws, device=None):
@@ -219,15 +234,16 @@ def max_over_ranks(values, ws, device=None):
     return [float(x) for x in t.cpu()]
 
 
-def job_throughput(flops_per_step, ranks, ms_per_step):
-    """Whole-job TFLOP/s: every rank processes one sequence per step."""
-    return flops_per_step * ranks / (ms_per_step * 1e-3) / 1e12
+def job_throughput(flops_per_step, sequences, ms_per_step):
+    """Whole-job TFLOP/s: `sequences` sequences of `flops_per_step` each per
+    step (one per GPU for replicas, one in all for a split ring)."""
+    return flops_per_step * sequences / (ms_per_step * 1e-3) / 1e12
 
 
 class Path:
     """Device buffers and the C-ABI calls of one hot-path step."""
 
-    def __init__(self, w, device, seed_offset=0):
+    def __init__(self, w, device, seed_offset=0, owned=None, group=None):
         import torch
 
         import long_context_multimodal_b200 as m
@@ -235,6 +251,10 @@ class Path:
         self.m = m
         self.w = w
         self.dev = device
+        # owned: the virtual ranks this GPU computes when the ring is split
+        # across GPUs (split.RankRange), or None for the whole ring
+        self.owned = owned
+        self.group = group
         N, P, hq, hkv, d = w.N, w.P, w.hq, w.hkv, w.d
         self.seg_len, self.seg_kind = mi.workload_layout(w)
         vis = mi.token_kinds(self.seg_len, self.seg_kind) == mi.VISUAL
@@ -255,30 +275,59 @@ class Path:
         self.scale = 1.0 / math.sqrt(d)
         self.launches_per_step = 2 + 4 + 1 + 3 + 4  # maps+counts, 4 gathers, fwd, bwd x3, 4 scatters
 
+    def _exchange(self, *tensors):
+        """Split ring: every GPU's owned rows of these rank-local tensors to
+        every GPU (NCCL all-gather); nothing for the whole ring on one GPU."""
+        if self.owned is None:
+            return
+        from long_context_multimodal_b200 import split
+
+        for t in tensors:
+            split.all_gather_rows(t, self.owned, self.group)
+
+    def _exchange_workspace(self):
+        if self.owned is None:
+            return
+        import torch.distributed as dist
+
+        from long_context_multimodal_b200 import split
+
+        w = self.w
+        C = w.N // (2 * w.P)
+        slab = w.hq * 2 * ((C + 127) // 128 * 128)
+        for arr in split.workspace_slabs(self.ws, w.P, w.hq, C):
+            own = arr[self.owned.begin * slab:self.owned.end * slab].contiguous()
+            dist.all_gather_into_tensor(arr, own, group=self.group)
+
     def step(self, stream, ev=None):
         m, w = self.m, self.w
         N, P = w.N, w.P
+        rk = {} if self.owned is None else {"rank_begin": self.owned.begin, "rank_end": self.owned.end}
         m.mmsp_shard(self.seg_len, self.seg_kind, N, P, self.l2g, self.g2l, self.mod, self.segid, self.counts,
                      stream=stream)
         for src, dst in ((self.q, self.ql), (self.k, self.kl), (self.v, self.vl), (self.do, self.dol)):
             m.mmsp_shard(None, None, N, P, src=src, dst=dst, row_bytes=src[0].numel() * 2, stream=stream)
         if ev is not None:
             ev[0].record(stream)
+        self._exchange(self.kl, self.vl)
         m.mmsp_attn_fwd(self.ql, self.kl, self.vl, N, P, w.hq, w.hkv, w.d, self.scale, 1, 0, P, None, self.lse,
-                        self.ol, m.MMSP_FINALIZE, stream=stream)
+                        self.ol, m.MMSP_FINALIZE, stream=stream, **rk)
         if ev is not None:
             ev[1].record(stream)
         # the backward's three stages (what mmsp_attn_bwd runs), so that the
         # dominant dK/dV kernel can be timed on its own
-        m.mmsp_attn_bwd_prepare(self.ol, self.dol, self.lse, N, P, w.hq, w.d, self.ws, self.ws_bytes, stream=stream)
+        m.mmsp_attn_bwd_prepare(self.ol, self.dol, self.lse, N, P, w.hq, w.d, self.ws, self.ws_bytes, stream=stream,
+                                **rk)
+        self._exchange_workspace()
+        self._exchange(self.ql, self.dol)
         if ev is not None:
             ev[2].record(stream)
         m.mmsp_attn_bwd_dkdv(self.ql, self.kl, self.vl, self.dol, N, P, w.hq, w.hkv, w.d, self.scale, 1, self.dkl,
-                             self.dvl, self.ws, self.ws_bytes, stream=stream)
+                             self.dvl, self.ws, self.ws_bytes, stream=stream, **rk)
         if ev is not None:
             ev[3].record(stream)
         m.mmsp_attn_bwd_dq(self.ql, self.kl, self.vl, self.dol, N, P, w.hq, w.hkv, w.d, self.scale, 1, self.dql, None,
-                           self.ws, self.ws_bytes, stream=stream)
+                           self.ws, self.ws_bytes, stream=stream, **rk)
         if ev is not None:
             ev[4].record(stream)
         for src, dst in ((self.ol, self.o), (self.dql, self.dq), (self.dkl, self.dk), (self.dvl, self.dv)):
@@ -286,11 +335,12 @@ class Path:
                          stream=stream)
 
 
-def document_forward(m, path, w, dev, stream, time_calls):
-    """Forward of the packed-document variant: the workload's N tokens as a
-    buffer of short videos (mmsp_inputs.packed_documents), every document's
-    attention causal and isolated. Algorithmic flops count the visible
-    pairs, 4 d Hq sum_docs L (L + 1) / 2."""
+def document_masked(m, path, w, dev, stream, time_calls, peak):
+    """Forward and backward of the packed-document variant: the workload's
+    N tokens as a buffer of short videos (mmsp_inputs.packed_documents),
+    every document's attention causal and isolated. Algorithmic flops count
+    the visible pairs, 4 d Hq sum_docs L (L + 1) / 2 for the forward and
+    2.5x that for the backward (prepare + dK/dV + dQ)."""
     import torch
 
     doc_len, _, _ = mi.packed_documents(w.N, 3000 + w.index)
@@ -298,12 +348,65 @@ def document_forward(m, path, w, dev, stream, time_calls):
     m.mmsp_doc_starts(doc_len, w.N, ds, stream=stream)
     L = doc_len.astype(np.float64)
     flops = 4.0 * w.d * w.hq * float((L * (L + 1) / 2).sum())
-    ms = time_calls(lambda: m.mmsp_attn_fwd(path.ql, path.kl, path.vl, w.N, w.P, w.hq, w.hkv, w.d, path.scale, 1, 0,
-                                            w.P, None, path.lse, path.ol, m.MMSP_FINALIZE, doc_start=ds,
-                                            stream=stream))
+    N, P = w.N, w.P
+
+    def fwd():
+        m.mmsp_attn_fwd(path.ql, path.kl, path.vl, N, P, w.hq, w.hkv, w.d, path.scale, 1, 0, P, None, path.lse,
+                        path.ol, m.MMSP_FINALIZE, doc_start=ds, stream=stream)
+
+    def bwd():
+        m.mmsp_attn_bwd_prepare(path.ol, path.dol, path.lse, N, P, w.hq, w.d, path.ws, path.ws_bytes, stream=stream)
+        m.mmsp_attn_bwd_dkdv(path.ql, path.kl, path.vl, path.dol, N, P, w.hq, w.hkv, w.d, path.scale, 1, path.dkl,
+                             path.dvl, path.ws, path.ws_bytes, doc_start=ds, stream=stream)
+        m.mmsp_attn_bwd_dq(path.ql, path.kl, path.vl, path.dol, N, P, w.hq, w.hkv, w.d, path.scale, 1, path.dql,
+                           None, path.ws, path.ws_bytes, doc_start=ds, stream=stream)
+
+    ms = time_calls(fwd)
+    bms = time_calls(bwd, reps=3)
     m.mmsp_device_status(stream)
-    return {"documents": int(doc_len.size), "mean_tokens": float(L.mean()), "ms": ms,
-            "algorithmic_flops": flops, "tflops": flops / (ms * 1e-3) / 1e12}
+    fwd_line = {"documents": int(doc_len.size), "mean_tokens": float(L.mean()), "ms": ms,
+                "algorithmic_flops": flops, "tflops": flops / (ms * 1e-3) / 1e12,
+                "frac_of_peak": flops / (ms * 1e-3) / 1e12 / peak}
+    bwd_line = {"documents": int(doc_len.size), "ms": bms, "algorithmic_flops": 2.5 * flops,
+                "tflops": 2.5 * flops / (bms * 1e-3) / 1e12, "frac_of_peak": 2.5 * flops / (bms * 1e-3) / 1e12 / peak}
+    return fwd_line, bwd_line
+
+
+def hbm_kernels(m, path, w, dev, stream, time_calls, hbm_peak):
+    """The bandwidth-bound kernels timed alone at the workload's size, as
+    achieved GB/s of their algorithmic bytes: the zigzag maps (two int32
+    maps, uint8 modality, int32 segment id: 13 B per token), the plain row
+    gather of Q (read + write, 2 * Hq * d * 2 B per token), and the
+    standalone LSE merge of two fp32 partials over every (row, head) of the
+    sequence (read 2 d + 2, write d + 1 fp32: 1,548 B per row-head at
+    d = 128)."""
+    import torch
+
+    N, P, hq, d = w.N, w.P, w.hq, w.d
+
+    def line(name, nbytes, ms):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"kernel": name, "bound": "hbm", "bytes_per_launch": nbytes, "ms": ms, "achieved": gbs,
+                "unit": "GB/s", "peak": hbm_peak, "frac": gbs / hbm_peak}
+
+    out = {}
+    ms = time_calls(lambda: m.mmsp_shard(path.seg_len, path.seg_kind, N, P, path.l2g, path.g2l, path.mod, path.segid,
+                                         None, stream=stream), reps=20)
+    out["shard_maps"] = line("shard_maps_kernel", 13.0 * N, ms)
+    ms = time_calls(lambda: m.mmsp_shard(None, None, N, P, src=path.q, dst=path.ql, row_bytes=hq * d * 2,
+                                         stream=stream), reps=10)
+    out["shard_gather_q"] = line("shard_rows_kernel (Q)", 2.0 * N * hq * d * 2, ms)
+    g = torch.Generator(device=dev).manual_seed(11)
+    oa = torch.randn((N, hq, d), device=dev, generator=g)
+    ob = torch.randn((N, hq, d), device=dev, generator=g)
+    la = torch.randn((N, hq), device=dev, generator=g)
+    lb = torch.randn((N, hq), device=dev, generator=g)
+    ms = time_calls(lambda: m.mmsp_lse_merge(oa, la, ob, lb, oa, la, N, hq, d, stream=stream), reps=10)
+    out["lse_merge"] = line("lse_merge_kernel<128> (in place)", float(N * hq * (3 * d * 4 + 3 * 4)), ms)
+    m.mmsp_device_status(stream)
+    del oa, ob, la, lb
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_gpu(args):
@@ -318,8 +421,17 @@ def run_gpu(args):
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
     w = mi.WORKLOADS[args.workload]
-    path = Path(w, dev, seed_offset=rank)
+    split_ring = ws > 1 and args.mode == "split"
+    owned = None
+    if split_ring:
+        from long_context_multimodal_b200 import split
+
+        owned = split.owned_ranks(w.P, ws, rank, w.N // (2 * w.P))
+    # a split ring computes one sequence (the same seed on every GPU); the
+    # replicas compute one independent sequence per GPU
+    path = Path(w, dev, seed_offset=0 if split_ring else rank, owned=owned)
     m = path.m
+    sequences = 1 if split_ring else ws
     stream = torch.cuda.current_stream(dev)
 
     def barrier():
@@ -351,7 +463,8 @@ def run_gpu(args):
     bwd_ms = float(np.mean([e[1].elapsed_time(e[4]) for e in evs]))
     dkdv_ms = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
     dq_ms = float(np.mean([e[3].elapsed_time(e[4]) for e in evs]))
-    ok = bool(torch.isfinite(path.dq.float()).all()) and bool(torch.isfinite(path.o.float()).all())
+    rows = slice(None) if owned is None else owned.rows  # the rank-local rows this GPU computed
+    ok = all(bool(torch.isfinite(t[rows].float()).all()) for t in (path.ol, path.dql, path.dkl, path.dvl))
 
     # ---------------- end to end through the C ABI with host buffers
     pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
@@ -399,24 +512,26 @@ def run_gpu(args):
         [ms_total, e2e_ms, fwd_ms, bwd_ms, dkdv_ms, dq_ms], ws, dev)
     ms_step = ms_total / args.steps
     flops = w.fwd_bwd_flops()
-    value = job_throughput(flops, ws, ms_step)
+    value = job_throughput(flops, sequences, ms_step)
+    per_gpu = sequences / ws  # share of one sequence's work each GPU does
     if rank == 0:
         peaks, src = load_peaks()
         peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
         # dominant kernel (ncu launch list): the dK/dV kernel; its algorithmic
         # work is the four GEMM-equivalents S^T, dP^T, dV, dK = 2x forward
-        dkdv_flops = 2.0 * w.fwd_flops()
+        dkdv_flops = 2.0 * w.fwd_flops() * per_gpu
         achieved = dkdv_flops / (dkdv_ms * 1e-3) / 1e12
         traffic = profiled_traffic(f"attn_bwd_dkdv_{w.name}.md", ["attn_bwd.cuh", "ptx.cuh"])
         hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         rope_bytes = 2.0 * w.N * w.hq * w.d * 2  # read + write of Q, bf16
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w, ws),
-            "fwd_tflops": w.fwd_flops() / (fwd_ms * 1e-3) / 1e12,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "strong" if split_ring else "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w, ws, args.mode),
+            "fwd_tflops": w.fwd_flops() * per_gpu / (fwd_ms * 1e-3) / 1e12,
             "fwd_bwd_tflops": value / ws,
-            "frac_of_bf16_peak": {"fwd": w.fwd_flops() / (fwd_ms * 1e-3) / 1e12 / peak,
+            "frac_of_bf16_peak": {"fwd": w.fwd_flops() * per_gpu / (fwd_ms * 1e-3) / 1e12 / peak,
                                   "fwd_bwd": value / ws / peak, "peak_tflops": peak,
                                   "peak_kind": f"bf16_tflops_sustained ({src})"},
             "roofline": {"kernel": "attn_bwd_dkdv_kernel (mmsp_attn_bwd_dkdv)",
@@ -424,11 +539,11 @@ def run_gpu(args):
                          "frac": achieved / peak, "traffic": traffic,
                          "algorithmic_flops_per_launch": dkdv_flops, "launch_ms": dkdv_ms,
                          "peak_source": f"MEASURED_PEAKS.json bf16_tflops_sustained ({src})"},
-            "bwd_tflops": 2.5 * w.fwd_flops() / (bwd_ms * 1e-3) / 1e12,
+            "bwd_tflops": 2.5 * w.fwd_flops() * per_gpu / (bwd_ms * 1e-3) / 1e12,
             "kernel_ms": {"attn_fwd": fwd_ms, "attn_bwd_dkdv": dkdv_ms, "attn_bwd_dq": dq_ms,
                           "bwd_total": bwd_ms},
-            "e2e": {"value": flops * ws / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
+            "e2e": {"value": flops * sequences / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "rope_gather": {"kernel": "shard_rope_kernel<128, half pairs> on Q, theta = 1e7", "bound": "hbm",
                             "achieved": rope_bytes / (rope_ms * 1e-3) / 1e9, "unit": "GB/s",
                             "peak": hbm_peak, "frac": rope_bytes / (rope_ms * 1e-3) / 1e9 / hbm_peak,
@@ -446,14 +561,19 @@ def run_gpu(args):
             line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                                     "sample": f"{args.ref_rows} random query rows x {w.hq} heads of {w.name}: "
                                               f"fp64 forward + dQ backward ({dt:.1f} s)"}
-        if ws == 1:
-            # packed documents (attention reset per document) over the same
-            # rank-local Q, K, V; measured last and guarded so that a problem
-            # here is reported in the line instead of losing it
-            try:
-                line["document_masked_fwd"] = document_forward(m, path, w, dev, stream, time_calls)
-            except Exception as exc:  # noqa: BLE001
-                line["document_masked_fwd"] = {"error": f"{type(exc).__name__}: {exc}"}
+        # rank 0 alone, after the timed steps (the other ranks wait at the
+        # final barrier): the bandwidth-bound kernels and the packed-document
+        # variant on rank 0's buffers, each guarded so that a problem here is
+        # reported in the line instead of losing it
+        try:
+            line.update(hbm_kernels(m, path, w, dev, stream, time_calls, hbm_peak))
+        except Exception as exc:  # noqa: BLE001
+            line["hbm_kernels_error"] = f"{type(exc).__name__}: {exc}"
+        try:
+            line["document_masked_fwd"], line["document_masked_bwd"] = document_masked(m, path, w, dev, stream,
+                                                                                       time_calls, peak)
+        except Exception as exc:  # noqa: BLE001
+            line["document_masked_fwd"] = {"error": f"{type(exc).__name__}: {exc}"}
         print(json.dumps(line), flush=True)
     if ws > 1:
         dist.barrier()
@@ -467,6 +587,9 @@ def main():
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="n512k", choices=list(mi.WORKLOADS))
+    ap.add_argument("--mode", default="split", choices=["split", "replicas"],
+                    help="N > 1 GPUs: split one sequence's virtual ranks over the GPUs (strong scaling), or run "
+                         "one independent sequence per GPU (weak scaling)")
     ap.add_argument("--impl", default="mmsp", choices=["mmsp", "reference"])
     ap.add_argument("--ref-rows", type=int, default=48)
     ap.add_argument("--e2e-steps", type=int, default=None)

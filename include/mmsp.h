@@ -23,8 +23,9 @@
  *     the calling thread's last error is available from mmsp_last_error().
  *   - All arguments are validated on the host before anything is launched;
  *     a rejected call launches nothing and touches no buffer.
- *   - Device pointers are caller-owned (the library allocates no device
- *     memory); host pointers are read during the call only.
+ *   - Device pointers are caller-owned (the library makes no runtime
+ *     allocation; its one piece of device memory is the fixed scratch of
+ *     mmsp_attn_bwd_noalloc); host pointers are read during the call only.
  *   - Work is enqueued asynchronously on `stream` (a cudaStream_t passed as
  *     void*; NULL means the legacy default stream). Nothing synchronises.
  *   - bf16 tensors are raw 16-bit bfloat16 words (const void*).
@@ -144,6 +145,14 @@ int mmsp_shard_rope(const void* src, void* dst, int64_t N, int32_t P,
  *   causal             1: key j visible to query i iff global j <= global i;
  *                      0: every key visible.
  *   step_begin/end     0 <= begin <= end <= P; (0, P) is the whole ring.
+ *   rank_begin/end     0 <= begin < end <= P: the virtual ranks whose queries
+ *                      this call computes; (0, P) is every rank. A GPU that
+ *                      owns a range of the ring's ranks (the ring split
+ *                      across GPUs, "MM-SP Mechanics", Ring-SP paragraph)
+ *                      computes its range after gathering every rank's K/V.
+ *                      All tensors keep their full [P][2C] shapes: q, o_acc,
+ *                      lse and o_out are read/written at the range's rows
+ *                      only; k and v are read at every rank's rows.
  *   o_acc              DEVICE fp32 [P][2C][Hq][d]: normalised output over the
  *                      keys seen so far. Read when flags has MMSP_ACCUMULATE,
  *                      written when non-NULL. Required with MMSP_ACCUMULATE.
@@ -167,6 +176,7 @@ int mmsp_attn_fwd(const void* q, const void* k, const void* v,
                   int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d,
                   float scale, int32_t causal,
                   int32_t step_begin, int32_t step_end,
+                  int32_t rank_begin, int32_t rank_end,
                   float* o_acc, float* lse, void* o_out,
                   uint32_t flags, const int32_t* doc_start, void* stream);
 
@@ -226,7 +236,11 @@ int mmsp_lse_merge(const float* o_a, const float* lse_a,
  *   workspace          DEVICE scratch of at least mmsp_bwd_workspace_bytes()
  *                      bytes (per-head LSE*log2(e) and D rows, about 8*Hq
  *                      bytes per token), 256-byte aligned; contents need not
- *                      be zeroed.
+ *                      be zeroed. Layout: two arrays (LSE*log2(e), then D,
+ *                      the second starting mmsp_bwd_workspace_bytes()/2
+ *                      bytes in), each fp32 [P][Hq][2][Cp] with Cp = C
+ *                      rounded up to a multiple of 128: rank r's rows are
+ *                      one contiguous slab of Hq*2*Cp floats per array.
  *   doc_start          as in mmsp_attn_fwd (the same array the forward used).
  *   d == 128 (MMSP_EUNSUPPORTED otherwise); other constraints as
  *   mmsp_attn_fwd.
@@ -252,18 +266,34 @@ int mmsp_attn_bwd(const void* q, const void* k, const void* v,
  * dkdv and dq read the prepared workspace and may run in either order. The
  * arguments mean what they mean for mmsp_attn_bwd; each call validates its
  * own and returns MMSP_EINVAL/MMSP_EUNSUPPORTED without launching.
+ *
+ * rank_begin/rank_end (0 <= begin < end <= P; (0, P) = every rank) select
+ * the virtual ranks a stage works for, so that a ring split across GPUs
+ * runs each stage on the ranks a GPU owns (tensors keep their full [P][2C]
+ * shapes, as in mmsp_attn_fwd):
+ *   prepare writes the workspace slabs of ranks [begin, end) from those
+ *           ranks' rows of o, dout and lse;
+ *   dq      writes dQ of the queries of ranks [begin, end); it reads those
+ *           ranks' q, dout and workspace slabs and every rank's k, v;
+ *   dkdv    writes dK, dV of the keys of ranks [begin, end); it reads those
+ *           ranks' k, v and EVERY rank's q, dout and workspace slabs (every
+ *           rank's queries may see the keys), so a split ring exchanges
+ *           q, dout and the prepared slabs before this stage.
  */
 int mmsp_attn_bwd_prepare(const void* o, const void* dout, const float* lse,
                           int64_t N, int32_t P, int32_t Hq, int32_t d,
+                          int32_t rank_begin, int32_t rank_end,
                           void* workspace, size_t workspace_bytes, void* stream);
 int mmsp_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout,
                        int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d,
-                       float scale, int32_t causal, void* dk, void* dv,
+                       float scale, int32_t causal, int32_t rank_begin, int32_t rank_end,
+                       void* dk, void* dv,
                        const void* workspace, size_t workspace_bytes,
                        const int32_t* doc_start, void* stream);
 int mmsp_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dout,
                      int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d,
-                     float scale, int32_t causal, void* dq, float* dq_acc_opt,
+                     float scale, int32_t causal, int32_t rank_begin, int32_t rank_end,
+                     void* dq, float* dq_acc_opt,
                      const void* workspace, size_t workspace_bytes,
                      const int32_t* doc_start, void* stream);
 
@@ -293,9 +323,12 @@ size_t mmsp_bwd_workspace_bytes(int64_t N, int32_t P, int32_t Hq, int32_t d);
  *   Sizes whose mmsp_bwd_workspace_bytes() exceeds the capacity are
  *   rejected with MMSP_EINVAL (nothing launched); for example with Hq = 28
  *   N = 262,144 needs about 59 MB and fits, N = 524,288 does not.
- *   The first call on a device resolves the array's device address on that
- *   device (cudaGetSymbolAddress, with that device current); make that first
- *   call before any stream capture. Later calls on the device reuse it.
+ *   The call looks up the array's device address on the current device
+ *   (cudaGetSymbolAddress, with that device current) whenever `stream` is
+ *   not being captured, so a device reset between calls is harmless. Under
+ *   stream capture it reuses the address found by the last uncaptured call
+ *   on that device: make the first call on a device before any stream
+ *   capture (a first call under capture is rejected with MMSP_EINVAL).
  *   The call allocates nothing (no cudaMalloc, cudaFree or allocating
  *   library routine). All calls on a device share the one array and it keeps
  *   the previous call's contents; everything the kernels need zeroed is

@@ -41,8 +41,8 @@ _SIGS = {
     "mmsp_shard": ([c_void_p, c_void_p, c_int32, c_int64, c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
                     c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_void_p], c_int32),
     "mmsp_attn_fwd": ([c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32, c_int32, c_int32, c_float,
-                       c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_uint32, c_void_p, c_void_p],
-                      c_int32),
+                       c_int32, c_int32, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_uint32, c_void_p,
+                       c_void_p], c_int32),
     "mmsp_doc_starts": ([c_void_p, c_int32, c_int64, c_void_p, c_void_p], c_int32),
     "mmsp_shard_rope": ([c_void_p, c_void_p, c_int64, c_int32, c_int32, c_int32, ctypes.c_double, c_int32, c_void_p,
                          c_int32, c_void_p], c_int32),
@@ -51,12 +51,14 @@ _SIGS = {
     "mmsp_attn_bwd": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32,
                        c_int32, c_int32, c_float, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                        c_size_t, c_void_p, c_void_p], c_int32),
-    "mmsp_attn_bwd_prepare": ([c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32, c_int32, c_void_p, c_size_t,
-                               c_void_p], c_int32),
+    "mmsp_attn_bwd_prepare": ([c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32, c_int32, c_int32, c_int32,
+                               c_void_p, c_size_t, c_void_p], c_int32),
     "mmsp_attn_bwd_dkdv": ([c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32, c_int32, c_int32,
-                            c_float, c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p], c_int32),
+                            c_float, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p,
+                            c_void_p], c_int32),
     "mmsp_attn_bwd_dq": ([c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32, c_int32, c_int32,
-                          c_float, c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p], c_int32),
+                          c_float, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p,
+                          c_void_p], c_int32),
     "mmsp_bwd_workspace_bytes": ([c_int64, c_int32, c_int32, c_int32], c_size_t),
     "mmsp_attn_bwd_noalloc": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32,
                                c_int32, c_int32, c_int32, c_float, c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -132,11 +134,18 @@ def mmsp_shard(seg_len, seg_kind, N, P, local2global=None, global2local=None, mo
     return _check("mmsp_shard", rc)
 
 
+def _ranks(P, rank_begin, rank_end):
+    return int(rank_begin), int(P if rank_end is None else rank_end)
+
+
 def mmsp_attn_fwd(q, k, v, N, P, Hq, Hkv, d, scale, causal, step_begin, step_end, o_acc, lse, o_out,
-                  flags, doc_start=None, stream=None):
+                  flags, doc_start=None, stream=None, rank_begin=0, rank_end=None):
+    """Ring attention forward of the virtual ranks [rank_begin, rank_end)
+    (default: every rank) over ring steps [step_begin, step_end)."""
+    rb, re = _ranks(P, rank_begin, rank_end)
     rc = _lib.mmsp_attn_fwd(_ptr(q), _ptr(k), _ptr(v), int(N), int(P), int(Hq), int(Hkv), int(d), float(scale),
-                            int(causal), int(step_begin), int(step_end), _ptr(o_acc), _ptr(lse), _ptr(o_out),
-                            int(flags), _ptr(doc_start), _stream(stream))
+                            int(causal), int(step_begin), int(step_end), rb, re, _ptr(o_acc), _ptr(lse),
+                            _ptr(o_out), int(flags), _ptr(doc_start), _stream(stream))
     return _check("mmsp_attn_fwd", rc)
 
 
@@ -169,24 +178,28 @@ def mmsp_attn_bwd(q, k, v, o, dout, lse, N, P, Hq, Hkv, d, scale, causal, dq, dk
     return _check("mmsp_attn_bwd", rc)
 
 
-def mmsp_attn_bwd_prepare(o, dout, lse, N, P, Hq, d, workspace, workspace_bytes, stream=None):
-    rc = _lib.mmsp_attn_bwd_prepare(_ptr(o), _ptr(dout), _ptr(lse), int(N), int(P), int(Hq), int(d), _ptr(workspace),
-                                    int(workspace_bytes), _stream(stream))
+def mmsp_attn_bwd_prepare(o, dout, lse, N, P, Hq, d, workspace, workspace_bytes, stream=None, rank_begin=0,
+                          rank_end=None):
+    rb, re = _ranks(P, rank_begin, rank_end)
+    rc = _lib.mmsp_attn_bwd_prepare(_ptr(o), _ptr(dout), _ptr(lse), int(N), int(P), int(Hq), int(d), rb, re,
+                                    _ptr(workspace), int(workspace_bytes), _stream(stream))
     return _check("mmsp_attn_bwd_prepare", rc)
 
 
 def mmsp_attn_bwd_dkdv(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, dk, dv, workspace, workspace_bytes,
-                       doc_start=None, stream=None):
+                       doc_start=None, stream=None, rank_begin=0, rank_end=None):
+    rb, re = _ranks(P, rank_begin, rank_end)
     rc = _lib.mmsp_attn_bwd_dkdv(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), int(N), int(P), int(Hq), int(Hkv), int(d),
-                                 float(scale), int(causal), _ptr(dk), _ptr(dv), _ptr(workspace),
+                                 float(scale), int(causal), rb, re, _ptr(dk), _ptr(dv), _ptr(workspace),
                                  int(workspace_bytes), _ptr(doc_start), _stream(stream))
     return _check("mmsp_attn_bwd_dkdv", rc)
 
 
 def mmsp_attn_bwd_dq(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, dq, dq_acc_opt, workspace, workspace_bytes,
-                     doc_start=None, stream=None):
+                     doc_start=None, stream=None, rank_begin=0, rank_end=None):
+    rb, re = _ranks(P, rank_begin, rank_end)
     rc = _lib.mmsp_attn_bwd_dq(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), int(N), int(P), int(Hq), int(Hkv), int(d),
-                               float(scale), int(causal), _ptr(dq), _ptr(dq_acc_opt), _ptr(workspace),
+                               float(scale), int(causal), rb, re, _ptr(dq), _ptr(dq_acc_opt), _ptr(workspace),
                                int(workspace_bytes), _ptr(doc_start), _stream(stream))
     return _check("mmsp_attn_bwd_dq", rc)
 

@@ -48,6 +48,7 @@ constexpr int TILE = 128 * 128 * 2;   // 32 KB bf16 tile
 
 struct Params {
   int32_t P, Hq, Hkv, G;
+  int32_t rank_begin, n_ranks;  // virtual ranks of this launch: dQ of their queries, dK/dV of their keys
   int64_t C;        // chunk length
   int64_t Cp;       // chunk length padded to a multiple of 128 (LSE2/D rows)
   int32_t ntiles;   // 128-row tiles per chunk
@@ -56,8 +57,8 @@ struct Params {
   int64_t n_items;  // dQ kernel work items
   float scale_log2;
   float scale;
-  const float* lse2t;   // [Hq][P][2][Cp]: LSE * log2(e); +inf on padding
-  const float* dt;      // [Hq][P][2][Cp]: D; 0 on padding
+  const float* lse2t;   // [P][Hq][2][Cp]: LSE * log2(e); +inf on padding
+  const float* dt;      // [P][Hq][2][Cp]: D; 0 on padding
   __nv_bfloat16* dq;    // [N][Hq][d]
   float* dq_acc;        // [N][Hq][d] fp32 dQ or nullptr
   __nv_bfloat16* dk;    // [N][Hkv][d]
@@ -91,19 +92,21 @@ struct Unit {
 };
 
 __device__ __forceinline__ Unit decode_unit(const Params& p, int64_t idx) {
-  // groups of decreasing work: global key chunk 0 first
+  // groups of decreasing work over the launch's key ranks [b, b + n):
+  // chunk 0 of rank b + g for g < n, then chunk 1 of rank b + 2n-1-g (the
+  // whole ring visits global key chunk g as group g, chunk 0 first)
   const int64_t per_chunk = (int64_t)p.ntiles * p.Hkv;
-  const int gk = (int)(idx / per_chunk);
-  const int64_t w = idx - (int64_t)gk * per_chunk;
+  const int g = (int)(idx / per_chunk);
+  const int64_t w = idx - (int64_t)g * per_chunk;
   Unit u;
-  u.gk = gk;
-  if (gk < p.P) {
-    u.k = gk;
+  if (g < p.n_ranks) {
+    u.k = p.rank_begin + g;
     u.ck = 0;
   } else {
-    u.k = 2 * p.P - 1 - gk;
+    u.k = p.rank_begin + 2 * p.n_ranks - 1 - g;
     u.ck = 1;
   }
+  u.gk = u.ck ? 2 * p.P - 1 - u.k : u.k;
   u.kvh = (int)(w / p.ntiles);
   u.kt = (int)(w % p.ntiles);
   u.key0 = (int64_t)u.kt * BM;
@@ -315,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx_w(leader, q_full(st), TILE + 1024);
         for (int hf = 0; hf < 2; ++hf)
           tma_load_3d_w(leader, sQ0 + st * TILE + hf * HALF, &tmQ, q_full(st), hf * 64, it.h, (int)it.lrow0);
-        const int64_t vrow = (((int64_t)it.h * p.P + it.r) * 2 + it.qcur) * p.Cp + it.q0;
+        const int64_t vrow = (((int64_t)it.r * p.Hq + it.h) * 2 + it.qcur) * p.Cp + it.q0;
         bulk_load_w(leader, sVEC + st * 1024, p.lse2t + vrow, 512, q_full(st));
         bulk_load_w(leader, sVEC + st * 1024 + 512, p.dt + vrow, 512, q_full(st));
         mbar_wait(do_empty(st), (use & 1) ^ 1, abort_flag, cap);
@@ -566,16 +569,18 @@ struct QItem {
 };
 
 __device__ __forceinline__ QItem decode_qitem(const Params& p, int64_t idx) {
-  // groups of decreasing work: global query chunk 2P-1 first
+  // groups of decreasing work over the launch's query ranks [b, b + n):
+  // chunk 1 of rank b + g for g < n, then chunk 0 of rank b + 2n-1-g (the
+  // whole ring visits global query chunk 2P-1-g as group g)
   const int64_t per_group = (int64_t)p.ntiles * p.Hq;
   const int g = (int)(idx / per_group);
   const int64_t w = idx - (int64_t)g * per_group;
   QItem it;
-  if (g < p.P) {
-    it.r = g;
+  if (g < p.n_ranks) {
+    it.r = p.rank_begin + g;
     it.c = 1;
   } else {
-    it.r = 2 * p.P - 1 - g;
+    it.r = p.rank_begin + 2 * p.n_ranks - 1 - g;
     it.c = 0;
   }
   const int hg = (int)(w % p.G);
@@ -876,7 +881,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const QItem it = decode_qitem(p, idx);
       const int64_t qin = it.q0 + row;  // query row within its chunk
       // this row's LSE*log2(e) and D (padding rows: +inf and 0)
-      const int64_t vrow = (((int64_t)it.h * p.P + it.r) * 2 + it.c) * p.Cp + qin;
+      const int64_t vrow = (((int64_t)it.r * p.Hq + it.h) * 2 + it.c) * p.Cp + qin;
       const float lse2 = p.lse2t[vrow];
       const float dval = p.dt[vrow];
       const int64_t gq_row = (int64_t)(it.c ? 2 * p.P - 1 - it.r : it.r) * p.C + qin;
@@ -1003,23 +1008,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // D_i = sum_d dO_i * O_i (fp32) and LSE_i * log2(e), written per head into
-// the padded [Hq][P][2][Cp] layout (+inf / 0 on padding rows). One warp per
-// (row, head); 8-byte loads.
+// the padded, rank-major [P][Hq][2][Cp] layout (+inf / 0 on padding rows),
+// for the rows of virtual ranks [rank_begin, rank_begin + n_ranks) (each
+// rank's rows are one contiguous slab, so a GPU that owns a range of ranks
+// can exchange its slab whole). One warp per (row, head); 8-byte loads.
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                       const __nv_bfloat16* __restrict__ dout,
                                                       const float* __restrict__ lse, float* __restrict__ lse2t,
-                                                      float* __restrict__ dt, int32_t P, int32_t Hq, int64_t C,
-                                                      int64_t Cp) {
+                                                      float* __restrict__ dt, int32_t rank_begin, int32_t n_ranks,
+                                                      int32_t Hq, int64_t C, int64_t Cp) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const int64_t total = (int64_t)P * 2 * Cp * Hq;  // padded (row, head) pairs
+  const int64_t total = (int64_t)n_ranks * 2 * Cp * Hq;  // padded (row, head) pairs of the launch's ranks
   for (int64_t w = warp; w < total; w += nwarps) {
     const int h = (int)(w % Hq);
-    const int64_t pr = w / Hq;   // padded row: (r*2 + c)*Cp + t
+    const int64_t pr = w / Hq;   // padded row within the range: (r'*2 + c)*Cp + t
     const int64_t t = pr % Cp;
-    const int64_t rc = pr / Cp;  // r*2 + c
-    const int64_t out_idx = ((int64_t)h * P * 2 + rc) * Cp + t;
+    const int64_t rc = pr / Cp + 2 * (int64_t)rank_begin;  // r*2 + c
+    const int64_t out_idx = (((rc >> 1) * Hq + h) * 2 + (rc & 1)) * Cp + t;
     if (t >= C) {
       if (lane == 0) {
         lse2t[out_idx] = CUDART_INF_F;

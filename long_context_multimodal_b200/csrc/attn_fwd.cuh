@@ -15,6 +15,8 @@
 // tiles A and B) of one zigzag chunk of one virtual rank. Items are ordered
 // by decreasing causal work (q chunk 2P-1 first), then kv head, row block,
 // query head, so CTAs running together stream the same K/V tiles through L2.
+// A launch may cover a range of virtual ranks only (the ranks one GPU owns
+// when the ring is split across GPUs); it reads every rank's K/V.
 // The CTA visits the item's K/V tiles of 128 keys in ring order and skips
 // (chunk, tile) pairs the causal mask empties.
 //
@@ -64,6 +66,7 @@ constexpr int HALF = 128 * 128;  // bytes of one 128-row x 64-column bf16 half t
 
 struct Params {
   int32_t P, Hq, Hkv, G;
+  int32_t rank_begin, n_ranks;  // the virtual ranks this launch computes: [rank_begin, rank_begin + n_ranks)
   int64_t C;        // zigzag chunk length N / (2P)
   int32_t nblk;     // 256-row blocks per chunk
   int32_t causal, step_begin, step_end;
@@ -88,13 +91,15 @@ __device__ __forceinline__ Item decode_item(const Params& p, int64_t idx) {
   const int g = (int)(idx / per_group);
   const int64_t w = idx - (int64_t)g * per_group;
   Item it;
-  // group g works on global query chunk 2P-1-g: chunk 1 of rank g for g < P,
-  // chunk 0 of rank 2P-1-g otherwise.
-  if (g < p.P) {
-    it.r = g;
+  // groups in decreasing causal work over the launch's ranks [b, b + n):
+  // chunk 1 of rank b + g (global chunk 2P-1-b-g) for g < n, then chunk 0
+  // of rank b + 2n-1-g (global chunk b + 2n-1-g). The whole ring (b = 0,
+  // n = P) visits global query chunk 2P-1-g as group g.
+  if (g < p.n_ranks) {
+    it.r = p.rank_begin + g;
     it.c = 1;
   } else {
-    it.r = 2 * p.P - 1 - g;
+    it.r = p.rank_begin + 2 * p.n_ranks - 1 - g;
     it.c = 0;
   }
   const int hg = (int)(w % p.G);

@@ -1,7 +1,9 @@
 // mmsp.cu -- the C ABI of libmmsp.so (declared in include/mmsp.h): host-side
 // validation, TMA descriptor encoding and stream-ordered launches of the
 // sm_100a kernels. One translation unit so that every kernel shares the
-// device-side timeout flag. The library allocates no device memory.
+// device-side timeout flag. The library makes no runtime allocation; its
+// only device memory of its own is the fixed module-scope scratch of
+// mmsp_attn_bwd_noalloc.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -111,6 +113,12 @@ int check_common(int64_t N, int32_t P) {
   if (P < 1) return fail(MMSP_EINVAL, "P must be >= 1 (got %d)", P);
   if (N >= (int64_t(1) << 31)) return fail(MMSP_EINVAL, "N must be < 2^31 (got %lld)", (long long)N);
   if (N % (2 * (int64_t)P) != 0) return fail(MMSP_EINVAL, "N (%lld) must be divisible by 2P (%d)", (long long)N, 2 * P);
+  return MMSP_OK;
+}
+
+int check_ranks(int32_t P, int32_t rank_begin, int32_t rank_end) {
+  if (rank_begin < 0 || rank_end <= rank_begin || rank_end > P)
+    return fail(MMSP_EINVAL, "need 0 <= rank_begin < rank_end <= P (got %d, %d, P=%d)", rank_begin, rank_end, P);
   return MMSP_OK;
 }
 
@@ -332,10 +340,12 @@ int launch_fwd(int dev, int vi, int64_t grid, cudaStream_t st, const CUtensorMap
 extern "C" {
 
 int mmsp_attn_fwd(const void* q, const void* k, const void* v, int64_t N, int32_t P, int32_t Hq, int32_t Hkv,
-                  int32_t d, float scale, int32_t causal, int32_t step_begin, int32_t step_end, float* o_acc,
-                  float* lse, void* o_out, uint32_t flags, const int32_t* doc_start, void* stream) {
+                  int32_t d, float scale, int32_t causal, int32_t step_begin, int32_t step_end, int32_t rank_begin,
+                  int32_t rank_end, float* o_acc, float* lse, void* o_out, uint32_t flags, const int32_t* doc_start,
+                  void* stream) {
   int rc = check_common(N, P);
   if (rc) return rc;
+  if ((rc = check_ranks(P, rank_begin, rank_end))) return rc;
   if ((rc = check_heads(Hq, Hkv, d))) return rc;
   if (doc_start && causal != 1) return fail(MMSP_EINVAL, "doc_start needs causal = 1");
   if (doc_start && ((uintptr_t)doc_start & 3u)) return fail(MMSP_EINVAL, "doc_start must be 4-byte aligned");
@@ -359,6 +369,8 @@ int mmsp_attn_fwd(const void* q, const void* k, const void* v, int64_t N, int32_
     return rc;
   fwd::Params p;
   p.P = P;
+  p.rank_begin = rank_begin;
+  p.n_ranks = rank_end - rank_begin;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
@@ -369,7 +381,7 @@ int mmsp_attn_fwd(const void* q, const void* k, const void* v, int64_t N, int32_
   p.step_end = step_end;
   p.accumulate = (flags & MMSP_ACCUMULATE) ? 1 : 0;
   p.finalize = (flags & MMSP_FINALIZE) ? 1 : 0;
-  p.n_items = 2LL * P * p.nblk * Hq;
+  p.n_items = 2LL * p.n_ranks * p.nblk * Hq;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o_acc = o_acc;
   p.lse = lse;
@@ -456,9 +468,11 @@ extern "C" size_t mmsp_bwd_workspace_bytes(int64_t N, int32_t P, int32_t Hq, int
 namespace {
 // Shared checks of the backward stages (sizes, scale, workspace).
 int bwd_check(int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d, float scale, int32_t causal,
-              const void* workspace, size_t workspace_bytes, const int32_t* doc_start = nullptr) {
+              int32_t rank_begin, int32_t rank_end, const void* workspace, size_t workspace_bytes,
+              const int32_t* doc_start = nullptr) {
   int rc = check_common(N, P);
   if (rc) return rc;
+  if ((rc = check_ranks(P, rank_begin, rank_end))) return rc;
   if ((rc = check_heads(Hq, Hkv, d))) return rc;
   if (d != 128) return fail(MMSP_EUNSUPPORTED, "the backward supports d = 128 (got %d)", d);
   if (!(scale > 0.f) || !std::isfinite(scale)) return fail(MMSP_EINVAL, "scale must be finite and > 0");
@@ -482,7 +496,8 @@ bool all_aligned16(std::initializer_list<const void*> ps) {
 
 // Parameters and tensor maps of the two tcgen05 backward kernels.
 int bwd_setup(const void* q, const void* k, const void* v, const void* dout, int64_t N, int32_t P, int32_t Hq,
-              int32_t Hkv, int32_t d, float scale, int32_t causal, const void* workspace, bwd::Params* p,
+              int32_t Hkv, int32_t d, float scale, int32_t causal, int32_t rank_begin, int32_t rank_end,
+              const void* workspace, bwd::Params* p,
               CUtensorMap* tq, CUtensorMap* tk, CUtensorMap* tv, CUtensorMap* tdo, int* sms) {
   int dev, rc;
   if ((rc = current_device(&dev)) || (rc = device_sms(dev, sms)) || (rc = get_encode())) return rc;
@@ -493,6 +508,8 @@ int bwd_setup(const void* q, const void* k, const void* v, const void* dout, int
   const char* ws = static_cast<const char*>(workspace);
   *p = bwd::Params{};
   p->P = P;
+  p->rank_begin = rank_begin;
+  p->n_ranks = rank_end - rank_begin;
   p->Hq = Hq;
   p->Hkv = Hkv;
   p->G = Hq / Hkv;
@@ -500,8 +517,8 @@ int bwd_setup(const void* q, const void* k, const void* v, const void* dout, int
   p->Cp = Lw.Cp;
   p->ntiles = (int32_t)(Lw.Cp / 128);
   p->causal = causal;
-  p->n_units = 2LL * P * p->ntiles * Hkv;
-  p->n_items = 2LL * P * p->ntiles * Hq;
+  p->n_units = 2LL * p->n_ranks * p->ntiles * Hkv;
+  p->n_items = 2LL * p->n_ranks * p->ntiles * Hq;
   p->scale_log2 = scale * 1.4426950408889634f;
   p->scale = scale;
   p->lse2t = reinterpret_cast<const float*>(ws);
@@ -524,8 +541,9 @@ int bwd_setup(const void* q, const void* k, const void* v, const void* dout, int
 }  // namespace
 
 extern "C" int mmsp_attn_bwd_prepare(const void* o, const void* dout, const float* lse, int64_t N, int32_t P,
-                                     int32_t Hq, int32_t d, void* workspace, size_t workspace_bytes, void* stream) {
-  int rc = bwd_check(N, P, Hq, 1, d, 1.f, 1, workspace, workspace_bytes);
+                                     int32_t Hq, int32_t d, int32_t rank_begin, int32_t rank_end, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  int rc = bwd_check(N, P, Hq, 1, d, 1.f, 1, rank_begin, rank_end, workspace, workspace_bytes);
   if (rc) return rc;
   if (!o || !dout || !lse) return fail(MMSP_EINVAL, "o, dout and lse must be non-NULL");
   if (!all_aligned16({o, dout, lse})) return fail(MMSP_EINVAL, "all tensors must be 16-byte aligned");
@@ -534,21 +552,22 @@ extern "C" int mmsp_attn_bwd_prepare(const void* o, const void* dout, const floa
   if ((rc = current_device(&dev)) || (rc = device_sms(dev, &sms))) return rc;
   const BwdLayout Lw = bwd_layout(N, P, Hq, d);
   char* ws = static_cast<char*>(workspace);
-  const int64_t pre_warps = (int64_t)P * 2 * Lw.Cp * Hq;
+  const int64_t pre_warps = (int64_t)(rank_end - rank_begin) * 2 * Lw.Cp * Hq;
   int64_t pre_blocks = (pre_warps + 7) / 8;
   if (pre_blocks > 16LL * sms) pre_blocks = 16LL * sms;
   bwd::bwd_pre_kernel<<<(unsigned)pre_blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse,
-      reinterpret_cast<float*>(ws), reinterpret_cast<float*>(ws + Lw.vec_bytes), P, Hq, Lw.C, Lw.Cp);
+      reinterpret_cast<float*>(ws), reinterpret_cast<float*>(ws + Lw.vec_bytes), rank_begin, rank_end - rank_begin, Hq,
+      Lw.C, Lw.Cp);
   MMSP_CUDA(cudaGetLastError());
   return ok();
 }
 
 extern "C" int mmsp_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout, int64_t N,
                                   int32_t P, int32_t Hq, int32_t Hkv, int32_t d, float scale, int32_t causal,
-                                  void* dk, void* dv, const void* workspace, size_t workspace_bytes,
-                                  const int32_t* doc_start, void* stream) {
-  int rc = bwd_check(N, P, Hq, Hkv, d, scale, causal, workspace, workspace_bytes, doc_start);
+                                  int32_t rank_begin, int32_t rank_end, void* dk, void* dv, const void* workspace,
+                                  size_t workspace_bytes, const int32_t* doc_start, void* stream) {
+  int rc = bwd_check(N, P, Hq, Hkv, d, scale, causal, rank_begin, rank_end, workspace, workspace_bytes, doc_start);
   if (rc) return rc;
   if (!q || !k || !v || !dout || !dk || !dv) return fail(MMSP_EINVAL, "q, k, v, dout, dk, dv must be non-NULL");
   if (!all_aligned16({q, k, v, dout, dk, dv})) return fail(MMSP_EINVAL, "all tensors must be 16-byte aligned");
@@ -556,7 +575,8 @@ extern "C" int mmsp_attn_bwd_dkdv(const void* q, const void* k, const void* v, c
   bwd::Params p;
   CUtensorMap tq, tk, tv, tdo;
   int sms;
-  if ((rc = bwd_setup(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, workspace, &p, &tq, &tk, &tv, &tdo, &sms)))
+  if ((rc = bwd_setup(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, rank_begin, rank_end, workspace, &p, &tq, &tk,
+                      &tv, &tdo, &sms)))
     return rc;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
@@ -573,10 +593,10 @@ extern "C" int mmsp_attn_bwd_dkdv(const void* q, const void* k, const void* v, c
 }
 
 extern "C" int mmsp_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dout, int64_t N, int32_t P,
-                                int32_t Hq, int32_t Hkv, int32_t d, float scale, int32_t causal, void* dq,
-                                float* dq_acc_opt, const void* workspace, size_t workspace_bytes,
-                                const int32_t* doc_start, void* stream) {
-  int rc = bwd_check(N, P, Hq, Hkv, d, scale, causal, workspace, workspace_bytes, doc_start);
+                                int32_t Hq, int32_t Hkv, int32_t d, float scale, int32_t causal, int32_t rank_begin,
+                                int32_t rank_end, void* dq, float* dq_acc_opt, const void* workspace,
+                                size_t workspace_bytes, const int32_t* doc_start, void* stream) {
+  int rc = bwd_check(N, P, Hq, Hkv, d, scale, causal, rank_begin, rank_end, workspace, workspace_bytes, doc_start);
   if (rc) return rc;
   if (!q || !k || !v || !dout || !dq) return fail(MMSP_EINVAL, "q, k, v, dout, dq must be non-NULL");
   if (!all_aligned16({q, k, v, dout, dq, dq_acc_opt})) return fail(MMSP_EINVAL, "all tensors must be 16-byte aligned");
@@ -584,7 +604,8 @@ extern "C" int mmsp_attn_bwd_dq(const void* q, const void* k, const void* v, con
   bwd::Params p;
   CUtensorMap tq, tk, tv, tdo;
   int sms;
-  if ((rc = bwd_setup(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, workspace, &p, &tq, &tk, &tv, &tdo, &sms)))
+  if ((rc = bwd_setup(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, rank_begin, rank_end, workspace, &p, &tq, &tk,
+                      &tv, &tdo, &sms)))
     return rc;
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dq_acc = dq_acc_opt;
@@ -604,19 +625,19 @@ extern "C" int mmsp_attn_bwd(const void* q, const void* k, const void* v, const 
                              const float* lse, int64_t N, int32_t P, int32_t Hq, int32_t Hkv, int32_t d, float scale,
                              int32_t causal, void* dq, void* dk, void* dv, float* dq_acc_opt, void* workspace,
                              size_t workspace_bytes, const int32_t* doc_start, void* stream) {
-  int rc = bwd_check(N, P, Hq, Hkv, d, scale, causal, workspace, workspace_bytes, doc_start);
+  int rc = bwd_check(N, P, Hq, Hkv, d, scale, causal, 0, P, workspace, workspace_bytes, doc_start);
   if (rc) return rc;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv)
     return fail(MMSP_EINVAL, "q, k, v, o, dout, lse, dq, dk, dv must be non-NULL");
   if (!all_aligned16({q, k, v, o, dout, lse, dq, dk, dv, dq_acc_opt}))
     return fail(MMSP_EINVAL, "all tensors must be 16-byte aligned");
   if (N == 0) return ok();
-  if ((rc = mmsp_attn_bwd_prepare(o, dout, lse, N, P, Hq, d, workspace, workspace_bytes, stream))) return rc;
-  if ((rc = mmsp_attn_bwd_dkdv(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, dk, dv, workspace, workspace_bytes,
-                               doc_start, stream)))
+  if ((rc = mmsp_attn_bwd_prepare(o, dout, lse, N, P, Hq, d, 0, P, workspace, workspace_bytes, stream))) return rc;
+  if ((rc = mmsp_attn_bwd_dkdv(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, 0, P, dk, dv, workspace,
+                               workspace_bytes, doc_start, stream)))
     return rc;
-  return mmsp_attn_bwd_dq(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, dq, dq_acc_opt, workspace, workspace_bytes,
-                          doc_start, stream);
+  return mmsp_attn_bwd_dq(q, k, v, dout, N, P, Hq, Hkv, d, scale, causal, 0, P, dq, dq_acc_opt, workspace,
+                          workspace_bytes, doc_start, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -630,12 +651,21 @@ std::mutex g_scratch_mu;
 
 // Device address of g_bwd_scratch on the current device (host code only
 // sees a host-side stand-in for the symbol; passing that to a kernel would
-// be wrong). Resolved once per device.
-int scratch_address(int dev, void** out) {
+// be wrong). Looked up again on every call made outside stream capture, so
+// that a context torn down and re-created (cudaDeviceReset) cannot leave a
+// stale address behind; a call under capture reuses the address of the
+// last uncaptured call on the device (the lookup allocates nothing either
+// way).
+int scratch_address(int dev, cudaStream_t st, void** out) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(st, &cs);
+  if (e != cudaSuccess) return fail(MMSP_ECUDA, "cudaStreamIsCapturing failed: %s", cudaGetErrorString(e));
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (cs == cudaStreamCaptureStatusNone || !g_scratch_ptr[dev]) {
+    if (cs != cudaStreamCaptureStatusNone)
+      return fail(MMSP_EINVAL, "the first mmsp_attn_bwd_noalloc call on a device must not be under stream capture");
     void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_bwd_scratch);
+    e = cudaGetSymbolAddress(&p, g_bwd_scratch);
     if (e != cudaSuccess || p == nullptr)
       return fail(MMSP_ECUDA, "cudaGetSymbolAddress(scratch) failed: %s", cudaGetErrorString(e));
     g_scratch_ptr[dev] = p;
@@ -661,7 +691,7 @@ extern "C" int mmsp_attn_bwd_noalloc(const void* q, const void* k, const void* v
   int dev;
   if ((rc = current_device(&dev))) return rc;
   void* scratch = nullptr;
-  if ((rc = scratch_address(dev, &scratch))) return rc;
+  if ((rc = scratch_address(dev, static_cast<cudaStream_t>(stream), &scratch))) return rc;
   return mmsp_attn_bwd(q, k, v, o, dout, lse, N, P, Hq, Hkv, d, scale, causal, dq, dk, dv, dq_acc_opt, scratch,
                        (size_t)MMSP_NOALLOC_SCRATCH_BYTES, doc_start, stream);
 }

@@ -48,9 +48,26 @@ def test_attn_fwd_rejects_bad_arguments():
     for bad in [dict(N=4095), dict(N=4100, P=4), dict(P=0), dict(N=-2), dict(Hq=6, Hkv=4), dict(d=96),
                 dict(d=256), dict(step_begin=3, step_end=2), dict(step_end=5), dict(q=p + 8), dict(lse=None),
                 dict(scale=0.0), dict(scale=float("nan")), dict(causal=2), dict(flags=8),
-                dict(flags=m.MMSP_ACCUMULATE, o_acc=None), dict(o_out=None), dict(N=1 << 31, P=1)]:
+                dict(flags=m.MMSP_ACCUMULATE, o_acc=None), dict(o_out=None), dict(N=1 << 31, P=1),
+                dict(rank_begin=0, rank_end=0), dict(rank_begin=2, rank_end=1), dict(rank_begin=-1),
+                dict(rank_end=5)]:
         args = dict(ok, **bad)
         _einval(F, **args)
+
+
+def test_backward_stages_reject_bad_rank_ranges():
+    import long_context_multimodal_b200 as m
+
+    p = 1 << 20
+    N, P, hq, hkv, d = 4096, 4, 4, 4, 128
+    wsb = m.mmsp_bwd_workspace_bytes(N, P, hq, d)
+    for rb, re in ((0, 0), (3, 2), (-1, 2), (0, 5)):
+        msg = _einval(m.mmsp_attn_bwd_prepare, p, p, p, N, P, hq, d, p, wsb, rank_begin=rb, rank_end=re)
+        assert "rank_begin" in msg
+        _einval(m.mmsp_attn_bwd_dkdv, p, p, p, p, N, P, hq, hkv, d, 0.088, 1, p, p, p, wsb, rank_begin=rb,
+                rank_end=re)
+        _einval(m.mmsp_attn_bwd_dq, p, p, p, p, N, P, hq, hkv, d, 0.088, 1, p, None, p, wsb, rank_begin=rb,
+                rank_end=re)
 
 
 def test_shard_rejects_bad_arguments():
