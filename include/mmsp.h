@@ -219,6 +219,35 @@ int mmsp_lse_merge(const float* o_a, const float* lse_a,
                    int64_t rows, int32_t H, int32_t d, void* stream);
 
 /*
+ * mmsp_ulysses_transpose -- the local sequence <-> head transpose around the
+ * Ulysses all-to-all of 2-D MM-SP (P = P_u x P_r).
+ *
+ * Source: "LongVILA Guide" (aifetchly), section "MM-SP Mechanics"
+ * (Ulysses: sequence-sharded (B, N/P, H, D) to head-sharded (B, N, H/P, D)
+ * by one all_to_all; the intra-node Ulysses level of MM-SP) and section
+ * "Implementation", UlyssesAllToAll (split into P_u contiguous head groups,
+ * group j to rank j, received pieces concatenated along the sequence in
+ * rank order; the inverse splits the sequence and concatenates the heads;
+ * the backward of one is the other).
+ *
+ *   src, dst     DEVICE buffers, 16-byte aligned, not overlapping; rows of
+ *                row_bytes (one head vector; a multiple of 16 bytes).
+ *   S            tokens this rank holds (>= 0; 0 is a no-op, pointers
+ *                unchecked); H heads, H % P_u == 0;
+ *                Hl = H / P_u heads per group.
+ *   unpack == 0  pack: src [S][H] -> dst [P_u][S][Hl], dst[j][s][h'] =
+ *                src[s][j*Hl + h'] (the send buffer of the forward
+ *                all-to-all: block j goes to Ulysses rank j).
+ *   unpack == 1  unpack: src [P_u][S][Hl] -> dst [S][H], the inverse (the
+ *                receive buffer of the inverse all-to-all, block i from
+ *                rank i, back to this rank's tokens with all heads).
+ * Bit-exact byte moves; bandwidth-bound.
+ */
+int mmsp_ulysses_transpose(const void* src, void* dst, int64_t S, int32_t H,
+                           int32_t P_u, int64_t row_bytes, int32_t unpack,
+                           void* stream);
+
+/*
  * mmsp_attn_bwd -- gradients of the ring attention (whole ring, all P ranks).
  *
  * The pages give only the backward of the all-to-all transpose; this is a

@@ -28,6 +28,7 @@ from ._binding import (  # noqa: F401
     mmsp_selftest_bounded_wait,
     mmsp_shard,
     mmsp_shard_rope,
+    mmsp_ulysses_transpose,
     mmsp_version,
     exported_symbols,
 )

@@ -48,6 +48,7 @@ _SIGS = {
                          c_int32, c_void_p], c_int32),
     "mmsp_lse_merge": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32,
                         c_void_p], c_int32),
+    "mmsp_ulysses_transpose": ([c_void_p, c_void_p, c_int64, c_int32, c_int32, c_int64, c_int32, c_void_p], c_int32),
     "mmsp_attn_bwd": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32,
                        c_int32, c_int32, c_float, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                        c_size_t, c_void_p, c_void_p], c_int32),
@@ -167,6 +168,14 @@ def mmsp_lse_merge(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, H, d, stream=No
     rc = _lib.mmsp_lse_merge(_ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(o_out), _ptr(lse_out),
                              int(rows), int(H), int(d), _stream(stream))
     return _check("mmsp_lse_merge", rc)
+
+
+def mmsp_ulysses_transpose(src, dst, S, H, P_u, row_bytes, unpack=False, stream=None):
+    """Sequence <-> head transpose around the Ulysses all-to-all (see mmsp.h):
+    pack [S][H] -> [P_u][S][H/P_u], or unpack the inverse."""
+    rc = _lib.mmsp_ulysses_transpose(_ptr(src), _ptr(dst), int(S), int(H), int(P_u), int(row_bytes),
+                                     int(bool(unpack)), _stream(stream))
+    return _check("mmsp_ulysses_transpose", rc)
 
 
 def mmsp_attn_bwd(q, k, v, o, dout, lse, N, P, Hq, Hkv, d, scale, causal, dq, dk, dv, dq_acc_opt,

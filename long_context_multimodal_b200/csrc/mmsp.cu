@@ -22,6 +22,7 @@
 #include "attn_fwd.cuh"
 #include "attn_bwd.cuh"
 #include "rope.cuh"
+#include "ulysses.cuh"
 
 using namespace mmsp;
 
@@ -279,6 +280,31 @@ int mmsp_shard_rope(const void* src, void* dst, int64_t N, int32_t P, int32_t H,
     break;
   switch (d) { MMSP_ROPE(8) MMSP_ROPE(16) MMSP_ROPE(32) MMSP_ROPE(64) MMSP_ROPE(128) MMSP_ROPE(256) }
 #undef MMSP_ROPE
+  MMSP_CUDA(cudaGetLastError());
+  return ok();
+}
+
+int mmsp_ulysses_transpose(const void* src, void* dst, int64_t S, int32_t H, int32_t P_u, int64_t row_bytes,
+                           int32_t unpack, void* stream) {
+  if (S < 0) return fail(MMSP_EINVAL, "S must be >= 0 (got %lld)", (long long)S);
+  if (H < 1 || P_u < 1 || H % P_u) return fail(MMSP_EINVAL, "need H %% P_u == 0 with H, P_u >= 1 (H=%d P_u=%d)", H, P_u);
+  if (row_bytes <= 0 || row_bytes % 16) return fail(MMSP_EINVAL, "row_bytes must be a positive multiple of 16");
+  if (unpack != 0 && unpack != 1) return fail(MMSP_EINVAL, "unpack must be 0 or 1");
+  if (S == 0) return ok();
+  if (!src || !dst) return fail(MMSP_EINVAL, "src and dst must be non-NULL");
+  if (!aligned16(src) || !aligned16(dst)) return fail(MMSP_EINVAL, "src and dst must be 16-byte aligned");
+  const int64_t run = (int64_t)(H / P_u) * row_bytes;
+  if (S > (int64_t(1) << 40) / ((int64_t)H * row_bytes)) return fail(MMSP_EINVAL, "tensor too large");
+  const int64_t bytes = S * P_u * run;
+  const char* s0 = static_cast<const char*>(src);
+  const char* d0 = static_cast<const char*>(dst);
+  if (s0 < d0 + bytes && d0 < s0 + bytes) return fail(MMSP_EINVAL, "src and dst overlap");
+  int dev, sms, rc;
+  if ((rc = current_device(&dev)) || (rc = device_sms(dev, &sms))) return rc;
+  int64_t blocks = (S * P_u + 7) / 8;  // 8 warps (runs) per block
+  if (blocks > 16LL * sms) blocks = 16LL * sms;
+  ulysses_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(src), static_cast<uint4*>(dst), S, P_u, run / 16, unpack);
   MMSP_CUDA(cudaGetLastError());
   return ok();
 }
