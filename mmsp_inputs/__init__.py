@@ -184,12 +184,27 @@ def workload_tensors(w: Workload, device="cpu", with_dout: Optional[bool] = None
 
 
 def sample_rows(N: int, C: int, count: int, seed: int) -> np.ndarray:
-    """Seeded global query positions: `count` draws plus forced edges
-    (0, N-1 and every chunk start), sorted and unique."""
+    """Seeded global query positions: `count` distinct random positions
+    other than the forced edges (0, N-1 and every chunk start), plus those
+    edges; sorted."""
     import torch
 
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
-    r = torch.randint(0, N, (count,), generator=g).numpy().astype(np.int64)
-    forced = np.concatenate([[0, N - 1], np.arange(0, N, C, dtype=np.int64)])
-    return np.unique(np.concatenate([r, forced]))
+    forced = np.unique(np.concatenate([[0, N - 1], np.arange(0, N, C, dtype=np.int64)]))
+    free = np.setdiff1d(np.arange(N, dtype=np.int64), forced)
+    count = min(count, len(free))
+    r = free[torch.randperm(len(free), generator=g)[:count].numpy()]
+    return np.sort(np.concatenate([r, forced]))
+
+
+def sample_keys(N: int, window: int, count: int, seed: int) -> np.ndarray:
+    """Seeded key positions: `count` distinct positions drawn from the last
+    `window` of the sequence (always including N-1), sorted."""
+    import torch
+
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    window = min(window, N)
+    r = N - window + torch.randperm(window - 1, generator=g)[:max(0, count - 1)].numpy().astype(np.int64)
+    return np.sort(np.concatenate([r, [N - 1]]))

@@ -144,10 +144,25 @@ def _head_groups(hq, hkv):
     return [[h for h in range(hq) if kv_head(h, hq, hkv) == kh] for kh in range(hkv)]
 
 
-def _row_block(n_vec, jmax, budget=1 << 26):
+BLOCK_BUDGET = 1 << 25  # elements of one fp64 score matrix (memory bound only)
+
+
+def _row_block(n_vec, jmax, budget=BLOCK_BUDGET):
     """Rows per block so that a [rows * n_vec, jmax] fp64 score matrix stays
-    within `budget` elements (memory bound only)."""
+    within `budget` elements."""
     return max(1, budget // max(1, n_vec * jmax))
+
+
+def _sorted_block(sorted_rows, b0, n_vec, block=None):
+    """Number of rows of the next block starting at index b0 of ascending
+    `sorted_rows`: `block` if given, else as many as keep the block's score
+    matrix in budget (its last, largest row sets the key count)."""
+    if block:
+        return block
+    nb = min(_row_block(n_vec, int(sorted_rows[b0]) + 1), len(sorted_rows) - b0)
+    while nb > 1 and nb * n_vec * (int(sorted_rows[b0 + nb - 1]) + 1) > BLOCK_BUDGET:
+        nb = (nb + 1) // 2
+    return nb
 
 
 def attention_rows(q_rows, k, v, rows, scale=None, block=None, doc_start=None):
@@ -244,10 +259,10 @@ def attention_bwd_rows(q_rows, k, v, do_rows, rows, scale=None, block=None, doc_
         G = len(heads)
         K = _t(k[:jmax_all, kh])
         V = _t(v[:jmax_all, kh])
+        srows = rows[order]
         b0 = 0
         while b0 < R:
-            jb = int(rows[order[b0]]) + 1
-            nb = block or _row_block(G, jb)
+            nb = _sorted_block(srows, b0, G, block)
             sel = order[b0:b0 + nb]
             b0 += nb
             rr = rows[sel]

@@ -1,8 +1,8 @@
 """Ring-blockwise causal attention forward on the GPU (C ABI) against the
 fp64 oracle: whole outputs at small sizes (several tiles, ragged chunk
 tails, every GQA ratio used), per-ring-step partials, the unfused
-step-by-step path with the standalone merge, and sampled rows at the full
-workload sizes."""
+step-by-step path with the standalone merge. The full workload sizes are in
+test_gpu_full_size.py."""
 import math
 
 import numpy as np
@@ -118,37 +118,3 @@ def test_empty_sequence_is_a_noop():
     l = torch.zeros(64, device="cuda")
     m.mmsp_attn_fwd(x, x, x, 0, 4, 4, 4, 64, 0.125, 1, 0, 4, None, l, None, 0)
     m.mmsp_device_status()
-
-
-def _sampled(name, count):
-    w = mi.WORKLOADS[name]
-    q, k, v, _ = mi.workload_tensors(w, device="cuda", with_dout=False)
-    o, lse, o_out = _path(q, k, v, w.P)
-    rows = mi.sample_rows(w.N, w.C, count, 3000 + w.index)
-    ridx = torch.as_tensor(rows, device="cuda")
-    o_s = o[ridx].cpu().numpy()
-    l_s = lse[ridx].cpu().numpy()
-    del o, lse, o_out
-    qr = q[ridx].float().cpu().numpy()
-    kc = k.float().cpu().numpy()
-    vc = v.float().cpu().numpy()
-    del q, k, v
-    torch.cuda.empty_cache()
-    o_ref, lse_ref = A.attention_rows(qr, kc, vc, rows)
-    return compare_attention(o_s, l_s, o_ref, lse_ref, f"{name} sampled rows")
-
-
-def test_n32k_sampled_rows():
-    _sampled("n32k", 4096)
-
-
-def test_n128k_sampled_rows():
-    _sampled("n128k", 4096)
-
-
-def test_n512k_sampled_rows():
-    _sampled("n512k", 384)
-
-
-def test_n1m_sampled_rows():
-    _sampled("n1m", 256)

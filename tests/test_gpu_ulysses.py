@@ -36,9 +36,9 @@ def test_pack_and_unpack_match_the_oracle(S, H, P_u, width, dtype):
     back = torch.full_like(x, float("nan"))
     m.mmsp_ulysses_transpose(packed, back, S, H, P_u, rb, unpack=True)
     m.mmsp_device_status()
-    ref = U.pack(x.cpu().numpy(), P_u)
     bits = torch.int16 if dtype == torch.bfloat16 else torch.int32
-    assert torch.equal(packed.cpu().view(bits), torch.from_numpy(ref).view(bits))
+    ref = U.pack(x.cpu().view(bits).numpy(), P_u)  # the oracle moves the raw bit patterns
+    assert torch.equal(packed.cpu().view(bits), torch.from_numpy(ref))
     assert torch.equal(back.view(bits), x.view(bits))
 
 

@@ -61,3 +61,33 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     with pytest.raises(m.MmspError) as e:
         m.mmsp_attn_bwd_noalloc(x, x, x, x, x, x, N, P, hq, 4, 128, 0.088, 1, x, x, x, None)
     assert e.value.status == 1 and "scratch" in str(e.value)
+
+
+def test_noalloc_backward_with_documents_on_a_side_stream_matches_the_oracle():
+    """Packed documents (the document-masked kernels through the shared
+    scratch) on a stream other than the default one, compared directly with
+    the fp64 oracle."""
+    import numpy as np
+
+    from oracle import attention as A
+
+    m = lib()
+    N, P, hq, hkv, d = 2400, 4, 4, 2, 128
+    doc_len = np.array([1000, 1, 599, 800], np.int32)
+    _, q, k, v, do = inputs(N, hq, hkv, d, seed=93, with_dout=True)
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        ds = torch.empty(N, dtype=torch.int32, device="cuda")
+        m.mmsp_doc_starts(doc_len, N, ds, stream=side)
+        ql, kl, vl, dol = (shard_rows(x, N, P) for x in (q, k, v, do))
+        _, lse, o = run_forward(ql, kl, vl, P, doc_start=ds)
+        dq, dk, dv = (torch.full_like(x, float("nan")) for x in (ql, kl, vl))
+        m.mmsp_attn_bwd_noalloc(ql, kl, vl, o, dol, lse, N, P, hq, hkv, d, 1.0 / math.sqrt(d), 1, dq, dk, dv, None,
+                                doc_start=ds, stream=side)
+        m.mmsp_device_status(side)
+        got = {n: shard_rows(t, N, P, inverse=True).float().cpu().numpy() for n, t in (("dQ", dq), ("dK", dk),
+                                                                                   ("dV", dv))}
+    ref = A.causal_attention_bwd(*(x.float().cpu().numpy() for x in (q, k, v, do)),
+                                 doc_start=A.document_starts(doc_len))
+    for name in ("dQ", "dK", "dV"):
+        compare_grad(got[name], ref[name], f"noalloc with documents {name}")
