@@ -35,6 +35,7 @@
 #include <math_constants.h>
 
 #include "ptx.cuh"
+#include "ring.cuh"
 
 namespace mmsp {
 namespace bwd {
@@ -118,6 +119,7 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int64_t idx) {
 template <bool DOC>
 struct VisitIter {
   int k, P, gk, causal, G, kvh, s, qc, t, tmax, hg, ntiles;
+  RingList ring;  // DOC: the few query chunks that can see the unit's keys
   int64_t C, key0, qrow_base, kg0, kg1, qchunk0;
   const int32_t* doc_start;
   bool in_chunk;
@@ -149,6 +151,16 @@ struct VisitIter {
     doc_start = p.doc_start;
     kg0 = (int64_t)u.gk * p.C + u.key0;
     kg1 = (int64_t)u.gk * p.C + (u.key0 + BM - 1 < p.C - 1 ? u.key0 + BM - 1 : p.C - 1);
+    ring.n = -1;
+    if constexpr (DOC) {
+      // queries see the keys only from chunk gk on, and only while their
+      // document starts at or before the unit's last key: the visible query
+      // chunks are [gk, c1] (document starts are non-decreasing). At step s
+      // the keys' block sits on rank (k + s) mod P.
+      int c1 = gk;
+      while (c1 + 1 < 2 * P && c1 - gk < 4 && (int64_t)doc_start[(int64_t)(c1 + 1) * C] <= kg1) ++c1;
+      ring.build(gk, c1, P, k, 1, 0, P);
+    }
   }
 
   // Document test of the current query tile: false if every query's
@@ -181,14 +193,20 @@ struct VisitIter {
         if (t <= tmax) continue;
         in_chunk = false;
       }
-      if (s >= P) return false;
-      r = (k + s) % P;
-      qcur = qc;
-      const int gq = qc ? 2 * P - 1 - r : r;
-      if (++qc == 2) {
-        qc = 0;
-        ++s;
+      int sc;
+      if (DOC && ring.n >= 0) {
+        if (!ring.pop(sc, qcur)) return false;
+      } else {
+        if (s >= P) return false;
+        sc = s;
+        qcur = qc;
+        if (++qc == 2) {
+          qc = 0;
+          ++s;
+        }
       }
+      r = (k + sc) % P;
+      const int gq = qcur ? 2 * P - 1 - r : r;
       if (causal && gq < gk) continue;
       diag = causal && gq == gk;
       // diagonal: only query tiles that reach the tile's first key
@@ -598,6 +616,7 @@ __device__ __forceinline__ QItem decode_qitem(const Params& p, int64_t idx) {
 template <bool DOC>
 struct KVIter {
   int r, P, gq, causal, s, ck, t, tmax, ntiles;
+  RingList ring;  // DOC: the few chunks that can hold visible keys
   int64_t C, q0, base_row, kchunk0, lo_min, lo_max;
   bool in_chunk, diag;
   int64_t kv_row, kglob0;
@@ -623,30 +642,43 @@ struct KVIter {
       const int64_t g0 = (int64_t)gq * C;
       lo_min = p.doc_start[g0 + q0];
       lo_max = p.doc_start[g0 + (q0 + BM - 1 < C - 1 ? q0 + BM - 1 : C - 1)];
+      // only chunks [lo_min / C, gq] can hold visible keys; at step s the
+      // rank holds the K/V of rank (r - s) mod P
+      ring.build((int)(lo_min / C), gq, P, r, -1, 0, P);
+    } else {
+      ring.n = -1;
     }
   }
 
   __device__ __forceinline__ bool next() {
     while (true) {
       if (!in_chunk) {
-        if (s >= P) return false;
-        int k = (r - s) % P;
+        int sc, ckc;
+        if (DOC && ring.n >= 0) {
+          if (!ring.pop(sc, ckc)) return false;
+        } else {
+          if (s >= P) return false;
+          sc = s;
+          ckc = ck;
+          if (++ck == 2) {
+            ck = 0;
+            ++s;
+          }
+        }
+        int k = (r - sc) % P;
         if (k < 0) k += P;
-        const int gk = ck ? 2 * P - 1 - k : k;
+        const int gk = ckc ? 2 * P - 1 - k : k;
         const bool skip = causal && gk > gq;
         diag = causal && gk == gq;
-        base_row = (int64_t)k * 2 * C + (int64_t)ck * C;
+        base_row = (int64_t)k * 2 * C + (int64_t)ckc * C;
         kchunk0 = (int64_t)gk * C;
-        if (++ck == 2) {
-          ck = 0;
-          ++s;
-        }
         if (skip) continue;
         if (DOC && kchunk0 + C - 1 < lo_min) continue;  // whole chunk before every document
         int64_t last = q0 + BM - 1;
         if (last > C - 1) last = C - 1;
         tmax = diag ? (int)(last / BN) : ntiles - 1;
-        t = 0;
+        // tiles wholly before every row's document hold no visible key
+        t = (DOC && lo_min > kchunk0) ? (int)((lo_min - kchunk0) / BN) : 0;
         in_chunk = true;
       }
       if (t > tmax) {

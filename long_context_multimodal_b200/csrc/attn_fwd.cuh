@@ -47,6 +47,7 @@
 #include <type_traits>
 
 #include "ptx.cuh"
+#include "ring.cuh"
 
 namespace mmsp {
 namespace fwd {
@@ -118,6 +119,7 @@ __device__ __forceinline__ Item decode_item(const Params& p, int64_t idx) {
 template <bool DOC>
 struct TileIter {
   int r, P, gq, causal, s, se, ck, t, tmax, ntiles;
+  RingList ring;  // DOC: the few chunks that can hold visible keys
   int64_t C, rowA0, base_row;
   int32_t kchunk0;  // global position of the current K/V chunk (N < 2^31)
   bool validA, validB, in_chunk, diag;
@@ -158,24 +160,37 @@ struct TileIter {
         loB_min = p.doc_start[g0 + (int32_t)rowA0 + 128];
         loB_max = p.doc_start[g0 + b1];
       }
+      // keys before loA_min (<= loB_min) are invisible to every row: only
+      // chunks [loA_min / C, gq] can hold visible keys; at step s the rank
+      // holds the K/V of rank (r - s) mod P
+      ring.build(loA_min / (int32_t)C, gq, P, r, -1, s, se);
+    } else {
+      ring.n = -1;
     }
   }
 
   __device__ __forceinline__ bool next() {
     while (true) {
       if (!in_chunk) {
-        if (s >= se) return false;
-        int k = (r - s) % P;
+        int sc, ckc;
+        if (DOC && ring.n >= 0) {
+          if (!ring.pop(sc, ckc)) return false;
+        } else {
+          if (s >= se) return false;
+          sc = s;
+          ckc = ck;
+          if (++ck == 2) {
+            ck = 0;
+            ++s;
+          }
+        }
+        int k = (r - sc) % P;
         if (k < 0) k += P;
-        const int gk = ck ? 2 * P - 1 - k : k;
+        const int gk = ckc ? 2 * P - 1 - k : k;
         const bool skip = causal && gk > gq;
         diag = causal && gk == gq;
-        base_row = (int64_t)k * 2 * C + (int64_t)ck * C;
+        base_row = (int64_t)k * 2 * C + (int64_t)ckc * C;
         kchunk0 = gk * (int32_t)C;
-        if (++ck == 2) {
-          ck = 0;
-          ++s;
-        }
         if (skip) continue;
         // whole chunk before every row's document
         const int32_t klast_chunk = kchunk0 + (int32_t)C - 1;
@@ -183,7 +198,8 @@ struct TileIter {
         int64_t last = rowA0 + (validB ? 255 : 127);
         if (last > C - 1) last = C - 1;
         tmax = diag ? (int)(last / BN) : ntiles - 1;
-        t = 0;
+        // tiles wholly before every row's document hold no visible key
+        t = (DOC && loA_min > kchunk0) ? (int)((loA_min - kchunk0) / BN) : 0;
         in_chunk = true;
       }
       if (t > tmax) {
