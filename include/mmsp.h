@@ -98,6 +98,52 @@ int mmsp_shard(const int32_t* seg_len, const uint8_t* seg_kind, int32_t n_seg,
                void* stream);
 
 /*
+ * mmsp_shard_frames -- the frame-aligned, modality-balanced shard of the
+ * per-token encoder stage, and its re-shard map into the zigzag layout.
+ *
+ * Source: "LongVILA Guide" (aifetchly), section "Problem" (modality-
+ * switching boundaries leave one rank with pure text and another with dense
+ * visual patches, and the ranks stall in the collectives). Reading: every
+ * frame (visual segment) goes WHOLE to encoder rank floor(P * V_f / V), V_f =
+ * visual tokens before it, V = all visual tokens, so every rank holds a
+ * contiguous block of frames within one frame of the share V/P; text token
+ * number t (text counted alone, T in all) goes to rank floor(P * t / T). The
+ * encoder layout concatenates the ranks in order, each rank's frames'
+ * tokens (sequence order) then its text tokens (sequence order).
+ *
+ *   seg_len, seg_kind  HOST table as in mmsp_shard (required, sums to N).
+ *   N, P               as mmsp_shard.
+ *   global2enc         DEVICE int32[N] or NULL: encoder-layout row of each
+ *                      global token.
+ *   local2enc          DEVICE int32[N] or NULL: encoder-layout row that
+ *                      zigzag rank-local slot l holds, i.e.
+ *                      global2enc[local2global[l]]: mmsp_gather_rows with it
+ *                      moves the encoder's output into the attention layout
+ *                      (scatter: the gradient back).
+ *   enc_counts         DEVICE int32[P][2] or NULL: visual, text tokens of
+ *                      each encoder rank.
+ * Bit-exact integer work.
+ */
+int mmsp_shard_frames(const int32_t* seg_len, const uint8_t* seg_kind, int32_t n_seg,
+                      int64_t N, int32_t P, int32_t* global2enc, int32_t* local2enc,
+                      int32_t* enc_counts, void* stream);
+
+/*
+ * mmsp_gather_rows -- indexed row copy: dst[i] = src[index[i]] (scatter ==
+ * 0) or dst[index[i]] = src[i] (scatter == 1), for i < n_rows; the re-shard
+ * between the encoder layout and the zigzag layout (mmsp_shard_frames).
+ *
+ *   src, dst   DEVICE rows of row_bytes (a multiple of 16), 16-byte
+ *              aligned, not overlapping; n_rows rows each.
+ *   index      DEVICE int32[n_rows], a permutation of [0, n_rows) for the
+ *              scatter. An entry outside [0, n_rows) is skipped and
+ *              reported by mmsp_device_status() as MMSP_EINVAL.
+ * Bit-exact byte moves; bandwidth-bound.
+ */
+int mmsp_gather_rows(const void* src, void* dst, const int32_t* index,
+                     int64_t n_rows, int64_t row_bytes, int32_t scatter, void* stream);
+
+/*
  * mmsp_shard_rope -- the shard gather of Q or K rows with the rotary
  * position embedding applied on the way (inverse == 0), or the transposed
  * rotation applied while scattering gradient rows back (inverse != 0).

@@ -28,6 +28,8 @@ from ._binding import (  # noqa: F401
     mmsp_selftest_bounded_wait,
     mmsp_shard,
     mmsp_shard_rope,
+    mmsp_shard_frames,
+    mmsp_gather_rows,
     mmsp_ulysses_transpose,
     mmsp_version,
     exported_symbols,

@@ -48,6 +48,9 @@ _SIGS = {
                          c_int32, c_void_p], c_int32),
     "mmsp_lse_merge": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32,
                         c_void_p], c_int32),
+    "mmsp_shard_frames": ([c_void_p, c_void_p, c_int32, c_int64, c_int32, c_void_p, c_void_p, c_void_p, c_void_p],
+                          c_int32),
+    "mmsp_gather_rows": ([c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int32, c_void_p], c_int32),
     "mmsp_ulysses_transpose": ([c_void_p, c_void_p, c_int64, c_int32, c_int32, c_int64, c_int32, c_void_p], c_int32),
     "mmsp_attn_bwd": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_int32,
                        c_int32, c_int32, c_float, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -168,6 +171,23 @@ def mmsp_lse_merge(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, H, d, stream=No
     rc = _lib.mmsp_lse_merge(_ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(o_out), _ptr(lse_out),
                              int(rows), int(H), int(d), _stream(stream))
     return _check("mmsp_lse_merge", rc)
+
+
+def mmsp_shard_frames(seg_len, seg_kind, N, P, global2enc=None, local2enc=None, enc_counts=None, stream=None):
+    """Frame-aligned, modality-balanced encoder shard maps (see mmsp.h)."""
+    sl_arr = np.ascontiguousarray(np.asarray(seg_len, dtype=np.int32))
+    sk_arr = np.ascontiguousarray(np.asarray(seg_kind, dtype=np.uint8))
+    rc = _lib.mmsp_shard_frames(sl_arr.ctypes.data_as(c_void_p), sk_arr.ctypes.data_as(c_void_p), int(sl_arr.size),
+                                int(N), int(P), _ptr(global2enc), _ptr(local2enc), _ptr(enc_counts),
+                                _stream(stream))
+    return _check("mmsp_shard_frames", rc)
+
+
+def mmsp_gather_rows(src, dst, index, n_rows, row_bytes, scatter=False, stream=None):
+    """dst[i] = src[index[i]] (or the scatter dst[index[i]] = src[i])."""
+    rc = _lib.mmsp_gather_rows(_ptr(src), _ptr(dst), _ptr(index), int(n_rows), int(row_bytes), int(bool(scatter)),
+                               _stream(stream))
+    return _check("mmsp_gather_rows", rc)
 
 
 def mmsp_ulysses_transpose(src, dst, S, H, P_u, row_bytes, unpack=False, stream=None):

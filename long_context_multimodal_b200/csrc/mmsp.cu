@@ -239,6 +239,65 @@ int mmsp_doc_starts(const int32_t* doc_len, int32_t n_doc, int64_t N, int32_t* d
   return ok();
 }
 
+int mmsp_shard_frames(const int32_t* seg_len, const uint8_t* seg_kind, int32_t n_seg, int64_t N, int32_t P,
+                      int32_t* global2enc, int32_t* local2enc, int32_t* enc_counts, void* stream) {
+  int rc = check_common(N, P);
+  if (rc) return rc;
+  if (!seg_len || !seg_kind) return fail(MMSP_EINVAL, "seg_len and seg_kind must be non-NULL");
+  if (N > 0 && (n_seg < 1 || n_seg > MMSP_MAX_SEGMENTS))
+    return fail(MMSP_EINVAL, "n_seg must be in [1, %d] (got %d)", MMSP_MAX_SEGMENTS, n_seg);
+  if (((uintptr_t)global2enc | (uintptr_t)local2enc | (uintptr_t)enc_counts) & 3u)
+    return fail(MMSP_EINVAL, "outputs must be 4-byte aligned");
+  if (N == 0) return ok();
+  static SegTable tab;
+  static std::mutex tab_mu;
+  std::lock_guard<std::mutex> lk(tab_mu);
+  int64_t acc = 0;
+  tab.n = n_seg;
+  for (int i = 0; i < n_seg; ++i) {
+    if (seg_len[i] < 1) return fail(MMSP_EINVAL, "segment %d has length %d < 1", i, seg_len[i]);
+    if (seg_kind[i] > 1) return fail(MMSP_EINVAL, "segment %d has kind %d (0 text, 1 visual)", i, seg_kind[i]);
+    tab.start[i] = (int32_t)acc;
+    tab.kind[i] = seg_kind[i];
+    acc += seg_len[i];
+    if (acc > N) break;
+  }
+  if (acc != N) return fail(MMSP_EINVAL, "segment lengths sum to %lld, expected N=%lld", (long long)acc, (long long)N);
+  tab.start[n_seg] = (int32_t)N;
+  if (!global2enc && !local2enc && !enc_counts) return ok();
+  int dev, sms;
+  if ((rc = current_device(&dev)) || (rc = device_sms(dev, &sms))) return rc;
+  int64_t blocks = (N + 255) / 256;
+  if (blocks > 8LL * sms) blocks = 8LL * sms;
+  frame_maps_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(tab, (int32_t)N, P, global2enc,
+                                                                                      local2enc, enc_counts);
+  MMSP_CUDA(cudaGetLastError());
+  return ok();
+}
+
+int mmsp_gather_rows(const void* src, void* dst, const int32_t* index, int64_t n_rows, int64_t row_bytes,
+                     int32_t scatter, void* stream) {
+  if (n_rows < 0 || n_rows >= (int64_t(1) << 31)) return fail(MMSP_EINVAL, "n_rows must be in [0, 2^31)");
+  if (row_bytes <= 0 || row_bytes % 16) return fail(MMSP_EINVAL, "row_bytes must be a positive multiple of 16");
+  if (scatter != 0 && scatter != 1) return fail(MMSP_EINVAL, "scatter must be 0 or 1");
+  if (n_rows == 0) return ok();
+  if (!src || !dst || !index) return fail(MMSP_EINVAL, "src, dst and index must be non-NULL");
+  if (!aligned16(src) || !aligned16(dst) || ((uintptr_t)index & 3u))
+    return fail(MMSP_EINVAL, "src/dst must be 16-byte aligned and index 4-byte aligned");
+  const int64_t bytes = n_rows * row_bytes;
+  const char* s0 = static_cast<const char*>(src);
+  const char* d0 = static_cast<const char*>(dst);
+  if (s0 < d0 + bytes && d0 < s0 + bytes) return fail(MMSP_EINVAL, "src and dst overlap");
+  int dev, sms, rc;
+  if ((rc = current_device(&dev)) || (rc = device_sms(dev, &sms))) return rc;
+  int64_t blocks = (n_rows + 7) / 8;  // 8 warps (rows) per block
+  if (blocks > 16LL * sms) blocks = 16LL * sms;
+  gather_rows_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(src), static_cast<uint4*>(dst), index, n_rows, row_bytes / 16, scatter);
+  MMSP_CUDA(cudaGetLastError());
+  return ok();
+}
+
 int mmsp_shard_rope(const void* src, void* dst, int64_t N, int32_t P, int32_t H, int32_t d, double theta,
                     int32_t interleaved, const int32_t* doc_start, int32_t inverse, void* stream) {
   int rc = check_common(N, P);
@@ -436,6 +495,7 @@ int mmsp_device_status(void* stream) {
     const int zero = 0;
     MMSP_CUDA(cudaMemcpyToSymbol(g_timeout_flag, &zero, sizeof(int)));
     if (flag == 2) return fail(MMSP_ECUDA, "a kernel found its shared memory base misaligned and did nothing");
+    if (flag == 3) return fail(MMSP_EINVAL, "an index array held a value out of range (those rows were skipped)");
     return fail(MMSP_ETIMEOUT, "a bounded device-side wait gave up");
   }
   return ok();

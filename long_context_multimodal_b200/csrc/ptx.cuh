@@ -12,7 +12,8 @@ namespace mmsp {
 
 // Device-side error word, read and cleared by mmsp_device_status() on the
 // host: 1 = a bounded wait gave up, 2 = a kernel found its shared memory
-// layout unusable and returned without work.
+// layout unusable and returned without work, 3 = an index argument held a
+// value out of range (the row was skipped).
 __device__ int g_timeout_flag = 0;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

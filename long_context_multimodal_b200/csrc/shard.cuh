@@ -149,4 +149,125 @@ __global__ void __launch_bounds__(256) shard_rows_words_kernel(const uint32_t* _
   }
 }
 
+// ----------------------------------------------------------------------------
+// Frame-aligned, modality-balanced encoder shard ("LongVILA Guide" (aifetchly),
+// section "Problem": modality-switching boundaries leave one rank with pure
+// text and another with dense visual patches). Reading: frame f (a visual
+// segment) goes whole to encoder rank floor(P * V_f / V), V_f = visual tokens
+// before it; text token t (text tokens counted alone) to rank floor(P * t /
+// T); the encoder layout is rank 0's frames then its text, rank 1's frames
+// then its text, and so on. With vis_start(e) = V_f of rank e's first frame
+// (V when none) and txt_start(e) = ceil(e * T / P), a visual token with
+// visual index v on rank e sits at row txt_start(e) + v, and a text token
+// with text index t on rank e at row vis_start(e + 1) + t.
+
+// Visual tokens before each segment (s_vis[0..n], s_vis[n] = V), by a
+// block-wide scan over the table: each thread sums a contiguous run of
+// segments, thread 0 scans the run totals, each thread writes its run.
+__device__ __forceinline__ void visual_prefix(const SegTable& tab, const int32_t* s_start, int32_t* s_vis,
+                                              int32_t* s_part) {
+  const int n = tab.n;
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int a = threadIdx.x * per, b = min(n, a + per);
+  int32_t sum = 0;
+  for (int i = a; i < b; ++i) sum += tab.kind[i] ? s_start[i + 1] - s_start[i] : 0;
+  s_part[threadIdx.x] = sum;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int32_t acc = 0;
+    for (int i = 0; i < (int)blockDim.x; ++i) {
+      const int32_t x = s_part[i];
+      s_part[i] = acc;
+      acc += x;
+    }
+  }
+  __syncthreads();
+  int32_t acc = s_part[threadIdx.x];
+  for (int i = a; i < b; ++i) {
+    s_vis[i] = acc;
+    acc += tab.kind[i] ? s_start[i + 1] - s_start[i] : 0;
+  }
+  if (b == n && a < b) s_vis[n] = acc;
+  if (n == 0 && threadIdx.x == 0) s_vis[0] = 0;
+  __syncthreads();
+}
+
+struct FramePlan {
+  const int32_t* start;  // shared: segment starts
+  const int32_t* vis;    // shared: visual tokens before each segment
+  const uint8_t* kind;   // segment kinds
+  int n, P;
+  int32_t V, T;
+
+  // V_f of the first frame whose rank is >= x (V when there is none).
+  __device__ __forceinline__ int32_t vis_start(int x) const {
+    const int64_t X = ((int64_t)x * V + P - 1) / P;
+    int lo = 0, hi = n;  // first s with vis[s] >= X (vis[n] = V >= X)
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (vis[mid] >= X) hi = mid;
+      else lo = mid + 1;
+    }
+    return vis[lo];
+  }
+  __device__ __forceinline__ int32_t txt_start(int x) const {
+    return (int32_t)(((int64_t)x * T + P - 1) / P);
+  }
+  __device__ __forceinline__ int32_t row(int32_t g) const {
+    const int s = seg_of(start, n, g);
+    if (kind[s]) {
+      const int e = (int)(((int64_t)P * vis[s]) / V);
+      return txt_start(e) + vis[s] + (g - start[s]);
+    }
+    const int32_t t = g - vis[s];
+    const int e = (int)(((int64_t)P * t) / T);
+    return vis_start(e + 1) + t;
+  }
+};
+
+__global__ void __launch_bounds__(256) frame_maps_kernel(const __grid_constant__ SegTable tab, int32_t N, int32_t P,
+                                                         int32_t* __restrict__ global2enc,
+                                                         int32_t* __restrict__ local2enc,
+                                                         int32_t* __restrict__ counts) {
+  __shared__ int32_t s_start[kMaxSegments + 1];
+  __shared__ int32_t s_vis[kMaxSegments + 1];
+  __shared__ int32_t s_part[256];
+  for (int i = threadIdx.x; i <= tab.n; i += blockDim.x) s_start[i] = tab.start[i];
+  __syncthreads();
+  visual_prefix(tab, s_start, s_vis, s_part);
+  FramePlan fp{s_start, s_vis, tab.kind, tab.n, P, s_vis[tab.n], N - s_vis[tab.n]};
+  const int64_t C = N / (2 * P);
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < N; i += (int64_t)gridDim.x * blockDim.x) {
+    if (global2enc) global2enc[i] = fp.row((int32_t)i);
+    if (local2enc) local2enc[i] = fp.row((int32_t)zigzag_global(i, C, P));
+  }
+  if (counts && blockIdx.x == 0) {
+    for (int e = threadIdx.x; e < P; e += blockDim.x) {
+      counts[2 * e + 0] = fp.vis_start(e + 1) - fp.vis_start(e);
+      counts[2 * e + 1] = fp.txt_start(e + 1) - fp.txt_start(e);
+    }
+  }
+}
+
+// Indexed row copy: dst[i] = src[index[i]] (gather) or dst[index[i]] =
+// src[i] (scatter), rows of row_vec 16-byte vectors; one warp per row. An
+// index outside [0, n_rows) is skipped and recorded (error word 3).
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                          const int32_t* __restrict__ index, int64_t n_rows,
+                                                          int64_t row_vec, int scatter) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t i = warp; i < n_rows; i += nwarps) {
+    const int64_t j = __ldg(index + i);
+    if (j < 0 || j >= n_rows) {
+      if (lane == 0) atomicExch(&g_timeout_flag, 3);
+      continue;
+    }
+    const uint4* a = src + (scatter ? i : j) * row_vec;
+    uint4* b = dst + (scatter ? j : i) * row_vec;
+    for (int64_t k = lane; k < row_vec; k += 32) b[k] = __ldg(a + k);
+  }
+}
+
 }  // namespace mmsp
