@@ -521,7 +521,7 @@ def run_gpu(args):
         # work is the four GEMM-equivalents S^T, dP^T, dV, dK = 2x forward
         dkdv_flops = 2.0 * w.fwd_flops() * per_gpu
         achieved = dkdv_flops / (dkdv_ms * 1e-3) / 1e12
-        traffic = profiled_traffic(f"attn_bwd_dkdv_{w.name}.md", ["attn_bwd.cuh", "ptx.cuh"])
+        traffic = profiled_traffic(f"attn_bwd_dkdv_{w.name}.md", ["attn_bwd.cuh", "ptx.cuh", "ring.cuh"])
         hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         rope_bytes = 2.0 * w.N * w.hq * w.d * 2  # read + write of Q, bf16
         line = {
@@ -574,6 +574,18 @@ def run_gpu(args):
                                                                                        time_calls, peak)
         except Exception as exc:  # noqa: BLE001
             line["document_masked_fwd"] = {"error": f"{type(exc).__name__}: {exc}"}
+        mhz = (clocks or {}).get("sm_mhz")
+        if mhz:
+            # the sustained peak was measured at a different SM clock than
+            # the one under this run's power cap: per-clock fractions
+            # against the nominal dense bf16 peak (2,250 TFLOP/s at the
+            # 1,965 MHz maximum clock) take the clock out of the comparison
+            nominal_per_ghz = 2250.0 / 1.965
+            line["per_clock"] = {"sm_mhz": mhz, "nominal_bf16_tflops_per_ghz": nominal_per_ghz,
+                                 "fwd_tflops_per_ghz": line["fwd_tflops"] / (mhz / 1e3),
+                                 "fwd_bwd_tflops_per_ghz": line["fwd_bwd_tflops"] / (mhz / 1e3),
+                                 "fwd_frac": line["fwd_tflops"] / (mhz / 1e3) / nominal_per_ghz,
+                                 "fwd_bwd_frac": line["fwd_bwd_tflops"] / (mhz / 1e3) / nominal_per_ghz}
         print(json.dumps(line), flush=True)
     if ws > 1:
         dist.barrier()
