@@ -299,13 +299,17 @@ class Path:
             own = arr[self.owned.begin * slab:self.owned.end * slab].contiguous()
             dist.all_gather_into_tensor(arr, own, group=self.group)
 
-    def step(self, stream, ev=None):
+    def step(self, stream, ev=None, io=None):
+        """One hot-path step. io: (inputs q, k, v, dO; outputs O, dQ, dK,
+        dV) in global order, default this path's own buffers."""
         m, w = self.m, self.w
         N, P = w.N, w.P
+        q, k, v, do, o, dq, dk, dv = io if io is not None else (self.q, self.k, self.v, self.do, self.o, self.dq,
+                                                                  self.dk, self.dv)
         rk = {} if self.owned is None else {"rank_begin": self.owned.begin, "rank_end": self.owned.end}
         m.mmsp_shard(self.seg_len, self.seg_kind, N, P, self.l2g, self.g2l, self.mod, self.segid, self.counts,
                      stream=stream)
-        for src, dst in ((self.q, self.ql), (self.k, self.kl), (self.v, self.vl), (self.do, self.dol)):
+        for src, dst in ((q, self.ql), (k, self.kl), (v, self.vl), (do, self.dol)):
             m.mmsp_shard(None, None, N, P, src=src, dst=dst, row_bytes=src[0].numel() * 2, stream=stream)
         if ev is not None:
             ev[0].record(stream)
@@ -330,7 +334,7 @@ class Path:
                            self.ws, self.ws_bytes, stream=stream, **rk)
         if ev is not None:
             ev[4].record(stream)
-        for src, dst in ((self.ol, self.o), (self.dql, self.dq), (self.dkl, self.dk), (self.dvl, self.dv)):
+        for src, dst in ((self.ol, o), (self.dql, dq), (self.dkl, dk), (self.dvl, dv)):
             m.mmsp_shard(None, None, N, P, src=src, dst=dst, row_bytes=src[0].numel() * 2, inverse=True,
                          stream=stream)
 
@@ -466,28 +470,64 @@ def run_gpu(args):
     rows = slice(None) if owned is None else owned.rows  # the rank-local rows this GPU computed
     ok = all(bool(torch.isfinite(t[rows].float()).all()) for t in (path.ol, path.dql, path.dkl, path.dvl))
 
-    # ---------------- end to end through the C ABI with host buffers
+    # ---------------- end to end through the C ABI with host buffers: every
+    # step copies its inputs from pinned host memory and its outputs back,
+    # on a copy stream, double-buffered so that step i+1's inputs arrive
+    # and step i's outputs leave while step i+1 computes
     pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-    h_in = [pin(t) for t in (path.q, path.k, path.v, path.do)]
-    for h, t in zip(h_in, (path.q, path.k, path.v, path.do)):
+    dev_in = [(path.q, path.k, path.v, path.do), tuple(torch.empty_like(t) for t in (path.q, path.k, path.v, path.do))]
+    dev_out = [(path.o, path.dq, path.dk, path.dv), tuple(torch.empty_like(t) for t in (path.o, path.dq, path.dk,
+                                                                                         path.dv))]
+    h_in = [pin(t) for t in dev_in[0]]
+    for h, t in zip(h_in, dev_in[0]):
         h.copy_(t)
-    h_out = [pin(t) for t in (path.o, path.dq, path.dk, path.dv)]
+    h_out = [pin(t) for t in dev_out[0]]
     h2d = sum(t.numel() * t.element_size() for t in h_in)
     d2h = sum(t.numel() * t.element_size() for t in h_out)
     e_steps = max(1, args.e2e_steps if args.e2e_steps is not None else args.steps)
+    copy_stream = torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e_steps):
-        for h, t in zip(h_in, (path.q, path.k, path.v, path.do)):
-            t.copy_(h, non_blocking=True)
-        path.step(stream)
-        for h, t in zip(h_out, (path.o, path.dq, path.dk, path.dv)):
-            h.copy_(t, non_blocking=True)
+    copy_stream.wait_event(e0)
+
+    def h2d_copy(b):
+        with torch.cuda.stream(copy_stream):
+            for h, t in zip(h_in, dev_in[b]):
+                t.copy_(h, non_blocking=True)
+        done = ev()
+        done.record(copy_stream)
+        return done
+
+    inputs_ready = [h2d_copy(0), None]
+    step_done = [None, None]   # step that last read/wrote buffer set b
+    outputs_read = [None, None]
+    for i in range(e_steps):
+        b = i % 2
+        stream.wait_event(inputs_ready[b])
+        if outputs_read[b] is not None:
+            stream.wait_event(outputs_read[b])  # step i-2's outputs have left
+        path.step(stream, io=dev_in[b] + dev_out[b])
+        step_done[b] = ev()
+        step_done[b].record(stream)
+        if i + 1 < e_steps:
+            nb = 1 - b
+            if step_done[nb] is not None:
+                copy_stream.wait_event(step_done[nb])  # step i-1 has read its inputs
+            inputs_ready[nb] = h2d_copy(nb)
+        copy_stream.wait_event(step_done[b])
+        with torch.cuda.stream(copy_stream):
+            for h, t in zip(h_out, dev_out[b]):
+                h.copy_(t, non_blocking=True)
+        outputs_read[b] = ev()
+        outputs_read[b].record(copy_stream)
+    stream.wait_event(outputs_read[(e_steps - 1) % 2])
     e1.record(stream)
     barrier()
     e2e_ms = e0.elapsed_time(e1) / e_steps
     m.mmsp_device_status(stream)
+    del dev_in, dev_out
 
     # ---------------- the RoPE-fused shard gather of Q (theta = 1e7), timed
     # on its own next to the plain gather it replaces (not part of the step:
