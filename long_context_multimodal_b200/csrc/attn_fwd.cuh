@@ -23,14 +23,16 @@
 // Warp roles (384 threads = three warpgroups, one CTA per SM):
 //   warp 0      TMA producer: Q tiles A/B once per item, then K_j, V_j into
 //               a 5-stage ring of 128 x d bf16 tiles (128-byte swizzle).
-//   warp 1      MMA issuer (warp-uniform, one lane issues): S_X = Q_X K_j^T
-//               into TMEM, and O_X += P_X V_j with P_X read from TMEM (the
-//               softmax writes bf16 P over the S columns it has consumed);
-//               ping-pong order PV_A(j), S_A(j+1), PV_B(j), S_B(j+1) so the
-//               tensor core works on one tile while the softmax warps work
-//               on the other. tcgen05 MMAs of one thread run in issue order,
-//               so S_X(j+1) overwrites P_X(j) only after PV_X(j) read it.
-//   warps 2-3   idle (they complete the first warpgroup's register release).
+//   warp 1      MMA issuer for tile A, warp 2 for tile B (warp-uniform, one
+//               lane issues): S_X = Q_X K_j^T into TMEM, and O_X += P_X V_j
+//               with P_X read from TMEM (the softmax writes bf16 P over the
+//               S columns it has consumed), in the order PV_X(j), S_X(j+1),
+//               so the tensor core works on one tile while the softmax warps
+//               work on the other. tcgen05 MMAs of one thread run in issue
+//               order, so S_X(j+1) overwrites P_X(j) only after PV_X(j) read
+//               it. Without document masks an issue token (two named
+//               barriers) keeps the tiles' groups in the order A, B per step.
+//   warp 3      idle (it completes the first warpgroup's register release).
 //   warps 4-7   softmax for tile A, warps 8-11 for tile B: one thread per
 //               row (TMEM lane) holding its whole row of S in registers,
 //               fp32 online softmax in base 2, P written to TMEM as bf16,
@@ -55,7 +57,7 @@ namespace fwd {
 constexpr int BM = 128;      // query rows per tile
 constexpr int BN = 128;      // keys per tile
 constexpr int NSTAGE = 5;    // K/V ring stages
-constexpr int kThreads = 384;  // three warpgroups: TMA + MMA (+2 idle warps), softmax A, softmax B
+constexpr int kThreads = 384;  // three warpgroups: TMA + 2 MMA (+1 idle warp), softmax A, softmax B
 // Register split: the launch gives 168 per thread (384 x 168 <= 65,536);
 // the control warpgroup drops to kRegCtl and the softmax warpgroups rise to
 // kRegSoftmax, keeping 128 x kRegCtl + 256 x kRegSoftmax <= 384 x 168.
@@ -266,10 +268,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < NSTAGE; ++i) {
       mbar_init(kv_full(i), 1);
-      mbar_init(kv_empty(i), 1);
+      mbar_init(kv_empty(i), 2);  // one release per MMA issuer
     }
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    mbar_init(q_empty, 2);
     for (int x = 0; x < 2; ++x) {
       mbar_init(s_full(x), 1);
       mbar_init(s_free(x), 4);
@@ -336,120 +338,151 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(kv_full((int)(i % NSTAGE)), (uint32_t)((i / NSTAGE) & 1), &no_abort, cap);
       if (qcnt > 0) mbar_wait(q_full, (qcnt - 1) & 1, &no_abort, cap);
     }
-  } else if (warp == 1) {
-    // -------------------------------------------------------- MMA issuer
-    // The whole warp runs the (uniform) control flow and computes the
-    // descriptors; lane 0 issues the tcgen05 instructions.
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------- MMA issuers
+    // Warp 1 issues tile A's MMAs, warp 2 tile B's: S_X = Q_X K^T and
+    // O_X += P_X V, each issuer in its own order (PV_X(j), then S_X(j+1),
+    // which overwrites P_X(j) only after PV_X(j) has read it: one thread's
+    // tcgen05 MMAs run in issue order). While one issuer waits for its P or
+    // does its bookkeeping, the other's MMAs keep the tensor core busy. Each
+    // K/V stage and the Q tiles are released once by each issuer: a commit if
+    // it read them, a plain arrival once the stage has filled if its tile had
+    // nothing to do there. The whole warp runs the (uniform) control flow and
+    // computes the descriptors; lane 0 issues the tcgen05 instructions.
+    //
+    // Without document masks every item is a long run of K/V tiles, and two
+    // free-running issuers let the softmax groups drift into phase, where
+    // they contend for the exponential unit. There an issue token keeps the
+    // order A, B, A, B per K/V step: named barrier 1 passes it from A to B,
+    // barrier 2 from B back to A (64 threads each: both issuer warps). Items
+    // of packed documents are short; there the issuers run free.
     {
+      constexpr bool kOrdered = !DOC;
+      const int x = warp - 1;  // 0: tile A, 1: tile B
       const uint32_t leader = lane == 0 ? 1u : 0u;
       constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(BM, D, 0, 1);
-      const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
-      const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
-      // operand descriptors, computed once: Q tiles, and stage 0 of the K/V
-      // ring (stage s is (s * KT) >> 4 further)
-      const uint64_t dQ[2] = {desc_kmajor_sw128(sQ0), desc_kmajor_sw128(sQ1)};
+      const uint32_t tSx = tmem + (uint32_t)(x * 128);
+      const uint32_t tOx = tmem + 256u + (uint32_t)(x * D);
+      // operand descriptors, computed once: this issuer's Q tile, and stage 0
+      // of the K/V ring (stage s is (s * KT) >> 4 further)
+      const uint64_t dQx = desc_kmajor_sw128(x ? sQ1 : sQ0);
       const uint64_t dK0 = desc_kmajor_sw128(sKV);
       const uint64_t dV0 = desc_mnmajor_sw128(sKV, HALF);
-      const std::integral_constant<int, 0> kA{};
-      const std::integral_constant<int, 1> kB{};
+      const uint32_t bar_s_full = s_full(x), bar_s_free = s_free(x), bar_p_full = p_full(x);
+      const uint32_t bar_o_done = o_done(x), bar_o_free = o_free(x);
       uint32_t pos = 0;  // K/V ring position (stage pos % NSTAGE)
-      uint32_t qcnt = 0;
-      uint32_t s_cnt[2] = {0, 0}, pv_cnt[2] = {0, 0}, epi_cnt[2] = {0, 0};
+      uint32_t qcnt = 0, s_cnt = 0, pv_cnt = 0, epi_cnt = 0;
+      uint32_t groups = 0;  // K/V steps this issuer has passed the token for
+      bool first_pv = true;
 
+      // Both issuers walk the same items and K/V steps, so every token taken
+      // is passed and every named-barrier phase completes, abort included
+      // (an aborted wait returns at once and the walk goes on).
+      auto take_token = [&]() {
+        if constexpr (kOrdered) {
+          __syncwarp();
+          if (x == 0) {
+            if (groups > 0) asm volatile("bar.sync 2, 64;" ::: "memory");
+          } else {
+            asm volatile("bar.sync 1, 64;" ::: "memory");
+          }
+        }
+      };
+      auto pass_token = [&]() {
+        if constexpr (kOrdered) {
+          __syncwarp();
+          if (x == 0) asm volatile("bar.arrive 1, 64;" ::: "memory");
+          else asm volatile("bar.arrive 2, 64;" ::: "memory");
+          ++groups;
+        }
+      };
       auto wait_full = [&](uint32_t ps) {
         mbar_wait(kv_full((int)(ps % NSTAGE)), (ps / NSTAGE) & 1, abort_flag, cap);
-        tc_fence_after();
       };
-      bool first_pv[2] = {true, true};
-      // Waits and issues are split so that all of a group's waits (P ready,
-      // O free, S buffer free) come before its PV and next S, which then go
-      // to the tensor pipe back to back.
-      auto wait_s_free = [&](auto X) {  // the softmax has released S_X
-        constexpr int x = decltype(X)::value;
-        if (s_cnt[x] > 0) mbar_wait(s_free(x), (s_cnt[x] - 1) & 1, abort_flag, cap);
+      auto release = [&](uint32_t ps, bool used) {  // this issuer is done with stage ps
+        if (used) mma_commit_w(leader, kv_empty((int)(ps % NSTAGE)));
+        else if (leader) mbar_arrive(kv_empty((int)(ps % NSTAGE)));
       };
-      auto wait_p = [&](auto X) {  // P_X written; O_X free at an item's first PV
-        constexpr int x = decltype(X)::value;
-        mbar_wait(p_full(x), pv_cnt[x] & 1, abort_flag, cap);
-        if (first_pv[x] && epi_cnt[x] > 0) mbar_wait(o_free(x), (epi_cnt[x] - 1) & 1, abort_flag, cap);
+      auto wait_s_free = [&]() {  // the softmax has read S_X (and P_X was consumed)
+        if (s_cnt > 0) mbar_wait(bar_s_free, (s_cnt - 1) & 1, abort_flag, cap);
       };
-      auto mma_S = [&](auto X, uint32_t kpos) {  // S_X = Q_X K^T
-        constexpr int x = decltype(X)::value;
+      auto mma_S = [&](uint32_t kpos) {  // S_X = Q_X K^T
         const uint64_t dk = dK0 + (uint64_t)((kpos % NSTAGE) * (L::KT >> 4));
         if (leader) {
-          mma_ss_kblock<D / 16, HALF>(tS[x], dQ[x], dk, idS, 0u);
-          mma_commit(s_full(x));
+          mma_ss_kblock<D / 16, HALF>(tSx, dQx, dk, idS, 0u);
+          mma_commit(bar_s_full);
         }
-        ++s_cnt[x];
+        ++s_cnt;
       };
-      auto mma_PV = [&](auto X, uint32_t vpos) {  // O_X += P_X V
-        constexpr int x = decltype(X)::value;
+      auto mma_PV = [&](uint32_t vpos) {  // O_X += P_X V
         const uint64_t dv = dV0 + (uint64_t)((vpos % NSTAGE) * (L::KT >> 4));
         // P_X is in TMEM over the first 64 columns of S_X (8 columns = 16
         // keys per instruction)
         if (leader) {
-          mma_ts_kblock<BN / 16>(tO[x], tS[x], dv, idO, first_pv[x] ? 0u : 1u);
-          mma_commit(o_done(x));
+          mma_ts_kblock<BN / 16>(tOx, tSx, dv, idO, first_pv ? 0u : 1u);
+          mma_commit(bar_o_done);
         }
-        ++pv_cnt[x];
-        first_pv[x] = false;
+        ++pv_cnt;
+        first_pv = false;
       };
 
       for (int64_t idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
         const Item it = decode_item(p, idx);
         mbar_wait(q_full, qcnt & 1, abort_flag, cap);
         ++qcnt;
-        tc_fence_after();
-        first_pv[0] = first_pv[1] = true;
+        first_pv = true;
         TileIter<DOC> ti(p, it);
         bool has = ti.next();
+        bool act = false;
         if (has) {
+          act = x ? ti.actB : ti.actA;
           const uint32_t kpos = pos++;
           wait_full(kpos);
-          if (ti.actA) wait_s_free(kA);
-          if (ti.actB) wait_s_free(kB);
-          tc_fence_after();
-          if (ti.actA) mma_S(kA, kpos);
-          if (ti.actB) mma_S(kB, kpos);
-          mma_commit_w(leader, kv_empty((int)(kpos % NSTAGE)));
+          if (act) wait_s_free();
+          take_token();
+          if (act) {
+            tc_fence_after();
+            mma_S(kpos);
+          }
+          release(kpos, act);
+          pass_token();
         }
         while (has) {
-          const bool curA = ti.actA, curB = ti.actB;
+          const bool cur = act;
           const uint32_t vpos = pos++;
           wait_full(vpos);
-          // next tile's bookkeeping and K wait first, so that S_X of the
-          // next tile follows PV_X in the tensor pipe without a gap
+          // the next tile's bookkeeping and waits come first, so that
+          // S_X(j+1) follows PV_X(j) in the tensor pipe without a gap
           const bool has_next = ti.next();
+          const bool nxt = has_next && (x ? ti.actB : ti.actA);
           uint32_t kn = 0;
           if (has_next) {
             kn = pos++;
             wait_full(kn);
           }
-          const bool nA = has_next && ti.actA, nB = has_next && ti.actB;
-          if (curA || nA) {
-            if (curA) wait_p(kA);
-            if (nA) wait_s_free(kA);
-            tc_fence_after();
-            if (curA) mma_PV(kA, vpos);
-            if (nA) mma_S(kA, kn);
+          if (cur) {  // P_X written; O_X free at an item's first PV
+            mbar_wait(bar_p_full, pv_cnt & 1, abort_flag, cap);
+            if (first_pv && epi_cnt > 0) mbar_wait(bar_o_free, (epi_cnt - 1) & 1, abort_flag, cap);
           }
-          if (curB || nB) {
-            if (curB) wait_p(kB);
-            if (nB) wait_s_free(kB);
-            tc_fence_after();
-            if (curB) mma_PV(kB, vpos);
-          }
-          mma_commit_w(leader, kv_empty((int)(vpos % NSTAGE)));
-          if (has_next) {
-            if (nB) mma_S(kB, kn);
-            mma_commit_w(leader, kv_empty((int)(kn % NSTAGE)));
-          }
+          if (nxt) wait_s_free();
+          take_token();
+          tc_fence_after();
+          if (cur) mma_PV(vpos);
+          release(vpos, cur);
+          if (nxt) mma_S(kn);
+          if (has_next) release(kn, nxt);
+          pass_token();
+          act = nxt;
           has = has_next;
         }
         mma_commit_w(leader, q_empty);
-        if (!first_pv[0]) ++epi_cnt[0];
-        if (!first_pv[1]) ++epi_cnt[1];
+        if (!first_pv) ++epi_cnt;
+      }
+      if constexpr (kOrdered) {
+        // take tile B's last token, so that barrier 2 ends with no phase open
+        __syncwarp();
+        if (x == 0 && groups > 0) asm volatile("bar.sync 2, 64;" ::: "memory");
       }
     }
   }
