@@ -132,15 +132,26 @@ class ClockSampler:
 
 
 _KV_CACHE = {}
+PARITY_ROWS = 4096  # the seeded query rows the full-size parity tests check
+
+
+def parity_rows(w, count, part=0):
+    """`count` query positions spread evenly over the seeded 4,096-row sample
+    the full-size parity tests use (mmsp_inputs.sample_rows with seed
+    3000 + index, forced chunk starts included); `part` picks a different
+    interleaved subset."""
+    sample = mi.sample_rows(w.N, w.C, PARITY_ROWS, 3000 + w.index)
+    stride = max(1, len(sample) // max(1, count))
+    return np.sort(sample[(part % stride)::stride][:count])
 
 
 def cpu_sample_inputs(w, rows_count, seed):
     """Rows of the workload for the CPU oracle without building all of Q:
-    K, V whole and Q, dO at the sampled rows (same recipe and distribution,
-    CPU generator)."""
+    K, V whole and Q, dO at rows of the parity sample (same recipe and
+    distribution, CPU generator)."""
     import torch
 
-    rows = np.sort(np.random.default_rng(seed).choice(w.N, rows_count, replace=False))
+    rows = parity_rows(w, rows_count, seed)
     g = torch.Generator().manual_seed(2000 + w.index + seed)
     bf = lambda *s: torch.randn(s, generator=g).to(torch.bfloat16)
     if w.name not in _KV_CACHE:
@@ -151,7 +162,7 @@ def cpu_sample_inputs(w, rows_count, seed):
         k[vis] = k[vis] * 2
         _KV_CACHE[w.name] = (k.float().numpy(), v.float().numpy())
     kc, vc = _KV_CACHE[w.name]
-    qr, dor = bf(rows_count, w.hq, w.d), bf(rows_count, w.hq, w.d)
+    qr, dor = bf(len(rows), w.hq, w.d), bf(len(rows), w.hq, w.d)
     return rows, qr.float().numpy(), kc, vc, dor.float().numpy()
 
 
@@ -183,7 +194,9 @@ def run_reference(args):
         return 0
     w = mi.WORKLOADS[args.workload]
     rows = args.ref_rows
-    sample = f"{rows} random query rows x all {w.hq} heads of {w.name} (N={w.N}): forward + dQ backward in fp64"
+    sample = (f"{rows} query rows x all {w.hq} heads of {w.name} (N={w.N}), an interleaved subset of the "
+              f"{PARITY_ROWS} seeded rows the parity tests check (a different subset each step): forward + dQ "
+              f"backward in fp64")
     for i in range(args.warmup):
         oracle_sample(w, max(4, rows // 8), 100 + i)
     vals, secs = [], 0.0
@@ -593,14 +606,15 @@ def run_gpu(args):
             "outputs_finite": ok,
         }
         if ws == 1 and not args.no_cpu_baseline:
-            rows = np.sort(np.random.default_rng(7).choice(w.N, args.ref_rows, replace=False))
+            rows = parity_rows(w, args.ref_rows)
             ridx = torch.as_tensor(rows, device=dev)
             inp = (rows, path.q[ridx].float().cpu().numpy(), path.k.float().cpu().numpy(),
                    path.v.float().cpu().numpy(), path.do[ridx].float().cpu().numpy())
-            fl, dt, threads = oracle_sample(w, args.ref_rows, 7, inputs=inp)
+            fl, dt, threads = oracle_sample(w, len(rows), 7, inputs=inp)
             line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                                    "sample": f"{args.ref_rows} random query rows x {w.hq} heads of {w.name}: "
-                                              f"fp64 forward + dQ backward ({dt:.1f} s)"}
+                                    "sample": f"{len(rows)} of the {PARITY_ROWS} seeded parity rows (evenly "
+                                              f"spread) x {w.hq} heads of {w.name}: fp64 forward + dQ "
+                                              f"backward ({dt:.1f} s)"}
         # rank 0 alone, after the timed steps (the other ranks wait at the
         # final barrier): the bandwidth-bound kernels and the packed-document
         # variant on rank 0's buffers, each guarded so that a problem here is
@@ -643,7 +657,7 @@ def main():
                     help="N > 1 GPUs: split one sequence's virtual ranks over the GPUs (strong scaling), or run "
                          "one independent sequence per GPU (weak scaling)")
     ap.add_argument("--impl", default="mmsp", choices=["mmsp", "reference"])
-    ap.add_argument("--ref-rows", type=int, default=48)
+    ap.add_argument("--ref-rows", type=int, default=192)
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
