@@ -657,7 +657,7 @@ def main():
                     help="N > 1 GPUs: split one sequence's virtual ranks over the GPUs (strong scaling), or run "
                          "one independent sequence per GPU (weak scaling)")
     ap.add_argument("--impl", default="mmsp", choices=["mmsp", "reference"])
-    ap.add_argument("--ref-rows", type=int, default=192)
+    ap.add_argument("--ref-rows", type=int, default=384)
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
