@@ -36,8 +36,8 @@
 //   warps 4-7   softmax for tile A, warps 8-11 for tile B: one thread per
 //               row (TMEM lane) holding its whole row of S in registers,
 //               fp32 online softmax in base 2, P written to TMEM as bf16,
-//               lazy O rescale (only when the running max grows by more than
-//               2^8), epilogue O / l and LSE.
+//               the running max raised (and O rescaled) whenever a tile
+//               holds a larger score, epilogue O / l and LSE.
 // The first warpgroup gives registers to the two softmax warpgroups
 // (setmaxnreg), see kRegCtl / kRegSoftmax.
 // TMEM: S_A [0,128) S_B [128,256) O_A [256,256+d) O_B [256+d,256+2d).
@@ -559,7 +559,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           mxv[1] = max3f(mxv[1], __uint_as_float(sr[126]), __uint_as_float(sr[127]));
           const float mx = max3f(mxv[0], mxv[1], fmaxf(mxv[2], mxv[3]));
           const float mc = fmaxf(m, mx * sl2);
-          need = mc > m + 8.0f;
+          // Raise the running max whenever the tile holds a larger score,
+          // so that the row's largest probability is exactly 1 when it is
+          // rounded to bf16 for the PV product. Raising it only past a margin
+          // (fewer O rescales) leaves that dominant term up to 2^-9 off,
+          // which on rows with few visible keys alone exceeds the output
+          // tolerance.
+          need = mc > m;
           alpha = 1.f;
           if (need) {
             alpha = ex2_approx(m - mc);
