@@ -74,3 +74,24 @@ def test_reference_arm_other_ranks_exit_quietly():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "n4k",
                         "--steps", "1", "--warmup", "3"], capture_output=True, text=True, timeout=300, env=env)
     assert r.returncode == 0 and "{" not in r.stdout
+
+
+def test_cpu_baseline_rows_come_from_the_parity_sample():
+    """The oracle timed as the CPU baseline runs on rows of the seeded sample
+    the full-size parity tests check: a sorted subset of the requested size,
+    spread over the sequence, and a different subset for another part."""
+    import numpy as np
+
+    sys.path.insert(0, ROOT)
+    import bench
+    import mmsp_inputs as mi
+
+    w = mi.WORKLOADS["n128k"]
+    sample = mi.sample_rows(w.N, w.C, bench.PARITY_ROWS, 3000 + w.index)
+    a = bench.parity_rows(w, 384)
+    b = bench.parity_rows(w, 384, part=1)
+    assert len(a) == 384 and len(b) == 384
+    assert np.all(np.diff(a) > 0) and np.isin(a, sample).all() and np.isin(b, sample).all()
+    assert not np.array_equal(a, b)
+    assert a[0] < w.N // 8 and a[-1] > w.N - w.N // 8  # spread over the sequence
+    assert len(bench.parity_rows(w, 10 * len(sample))) == len(sample)  # at most the whole sample
