@@ -8,7 +8,7 @@ Bar (derived from the arithmetic): the result is the fp32 rotation rounded
 to bf16, so |gpu - exact| <= 2^-8 |exact| (half a bf16 ulp, relative) plus
 the fp32 error of a cos - b sin, bounded by 2^-16 of the pair's norm (cos
 and sin carry about 2^-21 absolute error); results near zero by
-cancellation are judged by the second term. Almost every element must also
+cancellation are bounded by the second term. Almost every element must also
 equal the oracle rounded to bf16 exactly."""
 import numpy as np
 import pytest
