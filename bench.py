@@ -406,10 +406,38 @@ def hbm_kernels(m, path, w, dev, stream, time_calls, hbm_peak):
         return {"kernel": name, "bound": "hbm", "bytes_per_launch": nbytes, "ms": ms, "achieved": gbs,
                 "unit": "GB/s", "peak": hbm_peak, "frac": gbs / hbm_peak}
 
+    def graph_ms(call, reps=20):
+        """Device time per launch of `call`, captured `reps` times in a CUDA
+        graph and replayed back to back (for launches shorter than the host
+        work of one call: there, back-to-back calls leave the GPU idle)."""
+        cs = torch.cuda.Stream(device=dev)
+        cs.wait_stream(torch.cuda.current_stream(dev))
+        call(cs)
+        torch.cuda.synchronize(dev)
+        gph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gph, stream=cs):
+            for _ in range(reps):
+                call(cs)
+        with torch.cuda.stream(cs):
+            gph.replay()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(cs)
+            gph.replay()
+            b.record(cs)
+        b.synchronize()
+        del gph
+        return a.elapsed_time(b) / reps
+
     out = {}
-    ms = time_calls(lambda: m.mmsp_shard(path.seg_len, path.seg_kind, N, P, path.l2g, path.g2l, path.mod, path.segid,
-                                         None, stream=stream), reps=20)
+    maps_call = lambda st: m.mmsp_shard(path.seg_len, path.seg_kind, N, P, path.l2g, path.g2l, path.mod, path.segid,
+                                        None, stream=st)
+    host_ms = time_calls(lambda: maps_call(stream), reps=20)
+    try:
+        ms, how = graph_ms(maps_call), "CUDA graph of 20 launches replayed back to back (device time)"
+    except Exception as exc:  # noqa: BLE001
+        ms, how = host_ms, f"events around 20 calls, host work included (graph capture failed: {type(exc).__name__})"
     out["shard_maps"] = line("shard_maps_kernel", 13.0 * N, ms)
+    out["shard_maps"].update(timing=how, ms_per_call_with_host=host_ms)
     ms = time_calls(lambda: m.mmsp_shard(None, None, N, P, src=path.q, dst=path.ql, row_bytes=hq * d * 2,
                                          stream=stream), reps=10)
     out["shard_gather_q"] = line("shard_rows_kernel (Q)", 2.0 * N * hq * d * 2, ms)
