@@ -37,7 +37,9 @@
 //               row (TMEM lane) holding its whole row of S in registers,
 //               fp32 online softmax in base 2, P written to TMEM as bf16,
 //               the running max raised (and O rescaled) whenever a tile
-//               holds a larger score, epilogue O / l and LSE.
+//               holds a larger score (with documents: past a 2^8 margin,
+//               the dominant term of O corrected in the epilogue),
+//               epilogue O / l and LSE.
 // The first warpgroup gives registers to the two softmax warpgroups
 // (setmaxnreg), see kRegCtl / kRegSoftmax.
 // TMEM: S_A [0,128) S_B [128,256) O_A [256,256+d) O_B [256+d,256+2d).
@@ -507,7 +509,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // first visible key (global position) of this row's document
       const int32_t gqrow = (it.c ? 2 * p.P - 1 - it.r : it.r) * (int32_t)p.C + (int32_t)rin;
       const int32_t lo_row = (DOC && rin < p.C) ? p.doc_start[gqrow] : 0;
-      float m = -CUDART_INF_F, l = 0.f;
+      // m: stored running max (log2 units); l: running sum of the fp32
+      // probabilities; mxg: the row's largest raw score so far (document
+      // build only, see the epilogue).
+      float m = -CUDART_INF_F, l = 0.f, mxg = -CUDART_INF_F;
       int n_pv = 0;
       TileIter<DOC> ti(p, it);
       while (ti.next()) {
@@ -559,13 +564,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           mxv[1] = max3f(mxv[1], __uint_as_float(sr[126]), __uint_as_float(sr[127]));
           const float mx = max3f(mxv[0], mxv[1], fmaxf(mxv[2], mxv[3]));
           const float mc = fmaxf(m, mx * sl2);
-          // Raise the running max whenever the tile holds a larger score,
-          // so that the row's largest probability is exactly 1 when it is
-          // rounded to bf16 for the PV product. Raising it only past a margin
-          // (fewer O rescales) leaves that dominant term up to 2^-9 off,
-          // which on rows with few visible keys alone exceeds the output
-          // tolerance.
-          need = mc > m;
+          // P is rounded to bf16 for the PV product, so the row's largest
+          // probability must be exactly 1 or have its rounding error taken
+          // out: otherwise that dominant term is up to 2^-9 off, which on
+          // rows with few visible keys alone exceeds the output tolerance.
+          // Without documents the max is raised whenever a tile holds a
+          // larger score (the largest probability is then exactly 1). With
+          // documents rows are short and that would rescale O at almost
+          // every tile, so the max is raised only past a 2^8 margin and the
+          // epilogue corrects the dominant term instead.
+          if constexpr (DOC) {
+            need = mc > m + 8.0f;
+            mxg = fmaxf(mxg, mx);
+          } else {
+            need = mc > m;
+          }
           alpha = 1.f;
           if (need) {
             alpha = ex2_approx(m - mc);
@@ -631,14 +644,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 
       // ---------------------------------------------------------- epilogue
-      // O = acc / l and LSE = (m + log2 l) ln 2, merged into the running
-      // state when accumulating; written 32 columns at a time.
+      // O = acc / (l + c) and LSE = (m + log2 l) ln 2, merged into the
+      // running state when accumulating; written 32 columns at a time.
+      // Document build: c is the bf16 rounding error of the row's largest
+      // probability, added to the normaliser of O only. The stored max never
+      // changes after the tile that holds the row's largest score (that tile
+      // either raised it to the score, or the score is within 2^8 of it, and
+      // so is every later tile's max), so that element was computed with the
+      // final shift: the same fma, exponential and rounding as the tile
+      // (pack_bf16x2_alu) reproduce it here. Without documents c = 0.
       const float LN2 = 0.6931471805599453f;
       float lse_new = -CUDART_INF_F;
       float inv = 0.f;
       if (l > 0.f) {
         lse_new = (m + log2f(l)) * LN2;
-        inv = 1.f / l;
+        float c = 0.f;
+        if constexpr (DOC) {
+          const float e = ex2_approx(fmaf(mxg, sl2, -m));
+          c = __uint_as_float((__float_as_uint(e) + 0x8000u) & 0xFFFF0000u) - e;
+        }
+        inv = 1.f / (l + c);
       }
       const bool row_ok = rin < p.C;
       const int64_t lrow = (int64_t)it.r * 2 * p.C + (int64_t)it.c * p.C + rin;

@@ -116,19 +116,26 @@ def test_forward_documents_accumulate_over_step_ranges():
     compare_attention(o, l, O, L, "doc fwd accumulate")
 
 
-def test_one_document_is_bitwise_the_plain_path():
-    """doc_start all zero selects the document kernels but masks nothing:
-    bit-identical to doc_start = NULL, forward and backward."""
+def test_one_document_matches_the_plain_path():
+    """doc_start all zero selects the document kernels but masks nothing. The
+    document forward raises the running max only past a 2^8 margin and
+    corrects the dominant term of O; the plain forward raises it at every
+    increase. So the two forwards differ only by the bf16 rounding of P: both
+    match the oracle, and their LSEs agree to 1e-5. Given the same forward
+    outputs, the document backward is bit-identical to the plain backward."""
     N, P, hq, hkv, d = 2560, 4, 4, 2, 128
     q, k, v, do = _tensors(N, hq, hkv, d, 5, with_dout=True)
     ds = _doc_start_dev([N], N)
     ql, kl, vl, dol = (shard_rows(x, N, P) for x in (q, k, v, do))
     a = run_forward(ql, kl, vl, P)
     b = run_forward(ql, kl, vl, P, doc_start=ds)
-    for x, y in zip(a, b):
-        assert torch.equal(x, y)
+    back = lambda x: shard_rows(x, N, P, inverse=True).float().cpu().numpy()
+    o_ref, lse_ref = A.causal_attention(*_cpu(q, k, v))
+    compare_attention(back(a[0]), back(a[1]), o_ref, lse_ref, "plain path")
+    compare_attention(back(b[0]), back(b[1]), o_ref, lse_ref, "one document")
+    assert float((a[1] - b[1]).abs().max()) <= 1e-5
     ga = run_backward(ql, kl, vl, a[2], dol, a[1], P, fp32_dq=True)
-    gb = run_backward(ql, kl, vl, b[2], dol, b[1], P, fp32_dq=True, doc_start=ds)
+    gb = run_backward(ql, kl, vl, a[2], dol, a[1], P, fp32_dq=True, doc_start=ds)
     for x, y in zip(ga, gb):
         assert torch.equal(x, y)
 
