@@ -619,7 +619,8 @@ def run_gpu(args):
                          "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "algorithmic_flops_per_launch": dkdv_flops, "launch_ms": dkdv_ms,
-                         "peak_source": f"MEASURED_PEAKS.json bf16_tflops_sustained ({src})"},
+                         "peak_source": ("MEASURED_PEAKS.json bf16_tflops_sustained (measured)" if src == "measured"
+                                         else "profiling recipe fallback, bf16 sustained (no MEASURED_PEAKS.json)")},
             "bwd_tflops": 2.5 * w.fwd_flops() * per_gpu / (bwd_ms * 1e-3) / 1e12,
             "kernel_ms": {"attn_fwd": fwd_ms, "attn_bwd_dkdv": dkdv_ms, "attn_bwd_dq": dq_ms,
                           "bwd_total": bwd_ms},
